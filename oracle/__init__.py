@@ -1,0 +1,199 @@
+"""Float64 CPU oracle for block-sparse decode attention -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it and
+has no fallback to it.  The arithmetic lives in ``spattn_oracle.c`` (plain
+C, float64); this module only marshals numpy arrays into it.
+
+Every array argument is a numpy array holding the exact stored bytes:
+bf16 values as ``uint16`` bit patterns, fp8 e4m3fn values as ``uint8``
+codes, scales as ``float32``, tables and lengths as ``int32``.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "batch", "q_tokens", "num_q_heads", "num_kv_heads", "head_dim",
+        "block_size", "num_pages", "max_blocks", "max_sel", "kv_fp8")]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("sink_blocks", ctypes.c_int), ("local_blocks", ctypes.c_int),
+                ("mode", ctypes.c_int), ("top_k", ctypes.c_int),
+                ("top_p", ctypes.c_double), ("max_ratio", ctypes.c_double),
+                ("sm_scale", ctypes.c_double)]
+
+
+@dataclasses.dataclass
+class Dims:
+    batch: int
+    q_tokens: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_pages: int
+    max_blocks: int
+    max_sel: int
+    kv_fp8: bool = False
+
+    def c(self) -> _Dims:
+        return _Dims(self.batch, self.q_tokens, self.num_q_heads, self.num_kv_heads,
+                     self.head_dim, self.block_size, self.num_pages, self.max_blocks,
+                     self.max_sel, int(self.kv_fp8))
+
+
+@dataclasses.dataclass
+class Params:
+    sink_blocks: int = 1
+    local_blocks: int = 2
+    mode: str = "topk"          # "topk" | "topp"
+    top_k: int = 0
+    top_p: float = 1.0
+    max_ratio: float = 0.0
+    sm_scale: float = 0.0
+
+    def c(self) -> _Params:
+        return _Params(self.sink_blocks, self.local_blocks,
+                       0 if self.mode == "topk" else 1, self.top_k,
+                       float(self.top_p), float(self.max_ratio), float(self.sm_scale))
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        for name, args in {
+            "spo_compress_keys": [P, P, P, P, P, P],
+            "spo_block_scores": [P, P, P, P, P, P, P],
+            "spo_select": [P, P, P, P, P, P, P],
+            "spo_attend": [P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int, P],
+        }.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.spo_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.spo_bf16_to_f64.restype = ctypes.c_double
+        L.spo_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.spo_e4m3_to_f64.restype = ctypes.c_double
+        L.spo_num_threads.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_threads() -> int:
+    return lib().spo_num_threads()
+
+
+def bf16_to_f64(bits: int) -> float:
+    return lib().spo_bf16_to_f64(bits)
+
+
+def e4m3_to_f64(bits: int) -> float:
+    return lib().spo_e4m3_to_f64(bits)
+
+
+def _cache_dtype(dims: Dims):
+    return np.uint8 if dims.kv_fp8 else np.uint16
+
+
+def compress_keys(dims: Dims, k_cache, k_scale, block_table, seq_lens) -> np.ndarray:
+    """Mean-pooled key of every referenced block: float64 [num_pages][Hkv][d]."""
+    kbar = np.zeros((dims.num_pages, dims.num_kv_heads, dims.head_dim), np.float64)
+    k_cache = _c(k_cache, _cache_dtype(dims))
+    k_scale = _c(k_scale, np.float32) if dims.kv_fp8 else None
+    bt, sl = _c(block_table, np.int32), _c(seq_lens, np.int32)
+    rc = lib().spo_compress_keys(ctypes.byref(dims.c()), _ptr(k_cache), _ptr(k_scale),
+                                 _ptr(bt), _ptr(sl), _ptr(kbar))
+    if rc != 0:
+        raise ValueError(f"spo_compress_keys failed ({rc})")
+    return kbar
+
+
+def block_scores(dims: Dims, params: Params, q, kbar, block_table, seq_lens) -> np.ndarray:
+    """Block scores: float64 [B][Tq][Hkv][max_blocks], -inf outside the middle."""
+    s = np.empty((dims.batch, dims.q_tokens, dims.num_kv_heads, dims.max_blocks), np.float64)
+    q = _c(q, np.uint16)
+    kbar = _c(kbar, np.float64)
+    bt, sl = _c(block_table, np.int32), _c(seq_lens, np.int32)
+    rc = lib().spo_block_scores(ctypes.byref(dims.c()), ctypes.byref(params.c()), _ptr(q),
+                                _ptr(kbar), _ptr(bt), _ptr(sl), _ptr(s))
+    if rc != 0:
+        raise ValueError(f"spo_block_scores failed ({rc})")
+    return s
+
+
+def select(dims: Dims, params: Params, scores, seq_lens):
+    """Kept blocks per (b, h): (sel_idx [B][Hkv][max_sel], sel_count [B][Hkv], margin [B][Hkv])."""
+    sel = np.full((dims.batch, dims.num_kv_heads, dims.max_sel), -1, np.int32)
+    cnt = np.zeros((dims.batch, dims.num_kv_heads), np.int32)
+    margin = np.zeros((dims.batch, dims.num_kv_heads), np.float64)
+    scores = _c(scores, np.float64)
+    sl = _c(seq_lens, np.int32)
+    rc = lib().spo_select(ctypes.byref(dims.c()), ctypes.byref(params.c()), _ptr(scores),
+                          _ptr(sl), _ptr(sel), _ptr(cnt), _ptr(margin))
+    if rc != 0:
+        raise ValueError(f"spo_select failed ({rc}): max_sel too small")
+    return sel, cnt, margin
+
+
+def attend(dims: Dims, params: Params, q, k_cache, v_cache, k_scale, v_scale,
+           block_table, seq_lens, sel_idx, sel_count, units=None) -> np.ndarray:
+    """Softmax attention over the kept blocks: float64 [B][Tq][Hq][d].
+
+    ``units``: optional list of (b, h) pairs to compute; other rows stay 0.
+    """
+    out = np.zeros((dims.batch, dims.q_tokens, dims.num_q_heads, dims.head_dim), np.float64)
+    cd = _cache_dtype(dims)
+    k_cache, v_cache = _c(k_cache, cd), _c(v_cache, cd)
+    ks = _c(k_scale, np.float32) if dims.kv_fp8 else None
+    vs = _c(v_scale, np.float32) if dims.kv_fp8 else None
+    u = None if units is None else np.ascontiguousarray(np.asarray(units, np.int32).reshape(-1, 2))
+    rc = lib().spo_attend(ctypes.byref(dims.c()), ctypes.byref(params.c()), _ptr(_c(q, np.uint16)),
+                          _ptr(k_cache), _ptr(v_cache), _ptr(ks), _ptr(vs),
+                          _ptr(_c(block_table, np.int32)), _ptr(_c(seq_lens, np.int32)),
+                          _ptr(_c(sel_idx, np.int32)), _ptr(_c(sel_count, np.int32)),
+                          _ptr(u), 0 if u is None else len(u), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"spo_attend failed ({rc})")
+    return out
+
+
+def decode(dims: Dims, params: Params, q, k_cache, v_cache, k_scale, v_scale,
+           block_table, seq_lens, kbar=None, units=None):
+    """The whole path: compress (unless kbar given), score, select, attend.
+
+    Returns a dict with kbar, scores, sel_idx, sel_count, margin, out.
+    """
+    if kbar is None:
+        kbar = compress_keys(dims, k_cache, k_scale, block_table, seq_lens)
+    scores = block_scores(dims, params, q, kbar, block_table, seq_lens)
+    sel, cnt, margin = select(dims, params, scores, seq_lens)
+    out = attend(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table,
+                 seq_lens, sel, cnt, units)
+    return dict(kbar=kbar, scores=scores, sel_idx=sel, sel_count=cnt, margin=margin, out=out)
+
+
+__all__ = ["Dims", "Params", "compress_keys", "block_scores", "select", "attend", "decode",
+           "bf16_to_f64", "e4m3_to_f64", "num_threads", "lib"]

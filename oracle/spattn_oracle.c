@@ -1,0 +1,419 @@
+/*
+ * spattn_oracle.c -- float64 CPU oracle for block-sparse decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously-correct
+ * definition that the CUDA library is checked against.  Only the tests, the
+ * smoke check and the CPU-baseline leg of the benchmark load it.  It shares
+ * no source, header, table or helper with the CUDA library and must never be
+ * used as a fallback for it.
+ *
+ * What it computes, step by step, in float64 (sources are the pages this
+ * library restates; titles are given as printed on the pages):
+ *
+ *  1. Dequantise the stored cache.  bf16 is the upper half of an IEEE
+ *     binary32; fp8 e4m3fn is 1 sign / 4 exponent (bias 7) / 3 mantissa bits
+ *     with no infinities, times a per-(page, head) fp32 scale
+ *     ("Claude Code 1M 上下文", §2(3) "FP8量化与无损压缩": FP8 KV storage).
+ *  2. Block compression by mean pooling: one entry per 64-token block, the
+ *     mean of the keys of the tokens the block holds
+ *     ("Claude Code压缩上下文窗口的底层原理与性能优化实践", 算法流程, the
+ *     均值池化合并 node; "CSA + HCA 混合注意力机制" §4.1, where plain
+ *     averaging is named as the parameter-free compression).
+ *  3. Block scores: the query of each KV-head group, averaged over the group,
+ *     dotted with each compressed key and scaled by 1/sqrt(d)
+ *     ("CSA + HCA 混合注意力机制" §4.2 Lightning Indexer, steps 3-4, and
+ *     §4.4 step 1: score every compressed entry against the query).
+ *  4. Selection: the sink block and the local-window blocks are always kept;
+ *     the middle blocks are ranked by (score desc, index asc) and the top-k,
+ *     or the minimal top-p prefix of their softmax probabilities capped at
+ *     k_max, are kept ("Claude Opus 长上下文 KV Cache 稀疏注意力",
+ *     §稀疏注意力与 KV Cache 压缩的工程实现: block-level management,
+ *     attention sink, local context, Top-P selection; the configuration
+ *     table of §可落地的配置参数与监控要点; "CSA + HCA 混合注意力机制" §4.4
+ *     step 3 argsort/top-k).  For a chunk of query tokens the kept middle set
+ *     is the union over the tokens.
+ *  5. Exact softmax attention of every query head over every token of the
+ *     kept blocks, causal inside the chunk, scale 1/sqrt(d)
+ *     ("CSA + HCA 混合注意力机制" §2.1 scaled dot-product attention, §4.4
+ *     step 4).
+ *
+ * Where the pages are silent the reading taken is stated beside the code.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Keep in step with oracle/__init__.py (ctypes mirror). */
+typedef struct {
+    int batch;          /* B */
+    int q_tokens;       /* Tq: query tokens per request (1 = decode) */
+    int num_q_heads;    /* Hq */
+    int num_kv_heads;   /* Hkv; query head i reads KV head i / (Hq/Hkv) */
+    int head_dim;       /* d */
+    int block_size;     /* P: tokens per block (= per page) */
+    int num_pages;      /* pages in the cache pool */
+    int max_blocks;     /* columns of the block table */
+    int max_sel;        /* columns of the selection output */
+    int kv_fp8;         /* 0: bf16 cache, 1: fp8 e4m3fn cache + fp32 scales */
+} spo_dims;
+
+typedef struct {
+    int sink_blocks;    /* S */
+    int local_blocks;   /* W */
+    int mode;           /* 0: top-k, 1: top-p */
+    int top_k;          /* top-k: fixed k when > 0 */
+    double top_p;       /* top-p: mass threshold in (0, 1] */
+    double max_ratio;   /* cap k_max = floor(max_ratio * n_mid); <= 0: no cap */
+    double sm_scale;    /* 0: 1/sqrt(d) */
+} spo_params;
+
+/* ---------------------------------------------------------------- decoding */
+
+/* bf16 is the high 16 bits of a binary32: widening is exact. */
+double spo_bf16_to_f64(uint16_t bits)
+{
+    uint32_t w = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return (double)f;
+}
+
+/* e4m3fn: exponent bias 7, subnormals at exponent 0, S.1111.111 is NaN,
+ * no infinities. */
+double spo_e4m3_to_f64(uint8_t bits)
+{
+    int sign = (bits >> 7) & 1;
+    int e = (bits >> 3) & 0xF;
+    int m = bits & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Element (page, h, t, c) of a cache, dequantised. */
+static double cache_at(const spo_dims *dm, const void *cache, const float *scale,
+                       int64_t page, int h, int t, int c)
+{
+    int64_t off = (((page * dm->num_kv_heads + h) * dm->block_size) + t) * dm->head_dim + c;
+    if (dm->kv_fp8)
+        return spo_e4m3_to_f64(((const uint8_t *)cache)[off]) *
+               (double)scale[page * dm->num_kv_heads + h];
+    return spo_bf16_to_f64(((const uint16_t *)cache)[off]);
+}
+
+static int num_blocks(const spo_dims *dm, int len)
+{
+    return (len + dm->block_size - 1) / dm->block_size;
+}
+
+static double softmax_scale(const spo_dims *dm, const spo_params *pr)
+{
+    return pr->sm_scale > 0.0 ? pr->sm_scale : 1.0 / sqrt((double)dm->head_dim);
+}
+
+/* --------------------------------------------------------- 2. compression */
+
+/*
+ * kbar[page][h][c] = mean over the filled tokens of block j of K, for every
+ * block j of every request.  A block holds min(P, L - j*P) tokens; the tail
+ * block of a request is partly filled.  Pages not referenced are untouched.
+ */
+int spo_compress_keys(const spo_dims *dm, const void *k_cache, const float *k_scale,
+                      const int32_t *block_table, const int32_t *seq_lens,
+                      double *kbar)
+{
+    const int P = dm->block_size, D = dm->head_dim, H = dm->num_kv_heads;
+    for (int b = 0; b < dm->batch; ++b) {
+        int L = seq_lens[b];
+        int nb = num_blocks(dm, L);
+        if (nb > dm->max_blocks)
+            return -1;
+        #pragma omp parallel for schedule(dynamic)
+        for (int j = 0; j < nb; ++j) {
+            int64_t page = block_table[(int64_t)b * dm->max_blocks + j];
+            int filled = L - j * P < P ? L - j * P : P;
+            for (int h = 0; h < H; ++h)
+                for (int c = 0; c < D; ++c) {
+                    double s = 0.0;
+                    for (int t = 0; t < filled; ++t)
+                        s += cache_at(dm, k_cache, k_scale, page, h, t, c);
+                    kbar[(page * H + h) * D + c] = s / (double)filled;
+                }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------- 3. scores */
+
+/*
+ * scores[b][t][h][j] = scale * (qbar . kbar[page(b, j)][h]) for middle
+ * blocks j in [S, nb - W); -inf for every other column.  qbar is the mean of
+ * the G query rows that share KV head h (reading: the indexer aggregates
+ * over heads; with no learned indexer the group's mean query gives the mean
+ * of the group's per-head logits against the compressed key).
+ */
+int spo_block_scores(const spo_dims *dm, const spo_params *pr, const uint16_t *q,
+                     const double *kbar, const int32_t *block_table,
+                     const int32_t *seq_lens, double *scores)
+{
+    const int D = dm->head_dim, H = dm->num_kv_heads, Tq = dm->q_tokens;
+    const int G = dm->num_q_heads / H;
+    const double scale = softmax_scale(dm, pr);
+    const int64_t nrows = (int64_t)dm->batch * Tq * H;
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t row = 0; row < nrows; ++row) {
+        int h = (int)(row % H);
+        int t = (int)((row / H) % Tq);
+        int b = (int)(row / ((int64_t)H * Tq));
+        int nb = num_blocks(dm, seq_lens[b]);
+        double *out = scores + row * dm->max_blocks;
+        double *qbar = (double *)calloc((size_t)D, sizeof(double));
+        for (int g = 0; g < G; ++g)
+            for (int c = 0; c < D; ++c)
+                qbar[c] += spo_bf16_to_f64(
+                    q[(((int64_t)b * Tq + t) * dm->num_q_heads + h * G + g) * D + c]);
+        for (int c = 0; c < D; ++c)
+            qbar[c] /= (double)G;
+        for (int j = 0; j < dm->max_blocks; ++j) {
+            if (j < pr->sink_blocks || j >= nb - pr->local_blocks) {
+                out[j] = -INFINITY;
+                continue;
+            }
+            int64_t page = block_table[(int64_t)b * dm->max_blocks + j];
+            double s = 0.0;
+            for (int c = 0; c < D; ++c)
+                s += qbar[c] * kbar[(page * H + h) * D + c];
+            out[j] = s * scale;
+        }
+        free(qbar);
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------- 4. selection */
+
+typedef struct {
+    double s;
+    int j;
+} ranked;
+
+/* Rank order: higher score first; equal scores, lower block index first. */
+static int rank_cmp(const void *a, const void *b)
+{
+    const ranked *x = (const ranked *)a, *y = (const ranked *)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+/* Number of middle blocks kept for one query row, and the decision margin. */
+static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid,
+                          double *margin)
+{
+    int k_max = pr->max_ratio > 0.0 ? (int)floor(pr->max_ratio * (double)n_mid) : n_mid;
+    if (k_max > n_mid) k_max = n_mid;
+    double gap_inf = INFINITY;
+    *margin = gap_inf;
+    if (n_mid == 0)
+        return 0;
+    if (pr->mode == 0) {
+        /* top-k: k = top_k if given, else the ratio's k_max; never above the
+         * cap or the middle count. */
+        int k = pr->top_k > 0 ? pr->top_k : k_max;
+        if (k > k_max) k = k_max;
+        if (k > 0 && k < n_mid)
+            *margin = r[k - 1].s - r[k].s;
+        return k;
+    }
+    /* top-p: probabilities are the softmax of the middle scores; keep the
+     * minimal prefix of the ranked order whose mass reaches top_p
+     * (inclusive), then apply the cap. */
+    double mx = r[0].s, z = 0.0;
+    for (int i = 0; i < n_mid; ++i)
+        z += exp(r[i].s - mx);
+    double c = 0.0, c_prev = 0.0;
+    int m = n_mid;
+    for (int i = 0; i < n_mid; ++i) {
+        c_prev = c;
+        c += exp(r[i].s - mx) / z;
+        if (c >= pr->top_p) {
+            m = i + 1;
+            break;
+        }
+    }
+    if (m > k_max) {
+        /* the cap binds: the set is the top k_max; it would change only if
+         * the rank order at the cut changed or the mass at k_max reached p */
+        double cum = 0.0;
+        for (int i = 0; i < k_max; ++i)
+            cum += exp(r[i].s - mx) / z;
+        double mg = pr->top_p - cum;
+        if (k_max > 0 && k_max < n_mid && r[k_max - 1].s - r[k_max].s < mg)
+            mg = r[k_max - 1].s - r[k_max].s;
+        *margin = mg;
+        return k_max;
+    }
+    double mg = pr->top_p - c_prev;
+    if (m < n_mid && c - pr->top_p < mg && m < k_max)
+        mg = c - pr->top_p;
+    if (m < n_mid && r[m - 1].s - r[m].s < mg)
+        mg = r[m - 1].s - r[m].s;
+    *margin = mg;
+    return m;
+}
+
+/*
+ * Selection for every (b, h): sink blocks [0, S), local blocks [nb - W, nb)
+ * and, per query token t, the kept middle set M_t; the union over t is
+ * written ascending to sel_idx[b][h][*], its size to sel_count[b][h].
+ * margin[b][h] (optional) receives the smallest decision margin over t.
+ * Returns -2 if max_sel is too small for a row.
+ */
+int spo_select(const spo_dims *dm, const spo_params *pr, const double *scores,
+               const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_count,
+               double *margin)
+{
+    const int H = dm->num_kv_heads, Tq = dm->q_tokens;
+    int err = 0;
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t bh = 0; bh < (int64_t)dm->batch * H; ++bh) {
+        int b = (int)(bh / H), h = (int)(bh % H);
+        int nb = num_blocks(dm, seq_lens[b]);
+        int S = pr->sink_blocks, W = pr->local_blocks;
+        int n_mid = nb - S - W > 0 ? nb - S - W : 0;
+        char *keep = (char *)calloc((size_t)(nb > 0 ? nb : 1), 1);
+        ranked *r = (ranked *)malloc(sizeof(ranked) * (size_t)(n_mid > 0 ? n_mid : 1));
+        double mg_row = INFINITY;
+        for (int j = 0; j < nb; ++j)
+            if (j < S || j >= nb - W)
+                keep[j] = 1;
+        for (int t = 0; t < Tq; ++t) {
+            const double *s = scores + (((int64_t)b * Tq + t) * H + h) * dm->max_blocks;
+            for (int i = 0; i < n_mid; ++i) {
+                r[i].s = s[S + i];
+                r[i].j = S + i;
+            }
+            qsort(r, (size_t)n_mid, sizeof(ranked), rank_cmp);
+            double mg;
+            int m = row_keep_count(pr, r, n_mid, &mg);
+            if (mg < mg_row) mg_row = mg;
+            for (int i = 0; i < m; ++i)
+                keep[r[i].j] = 1;
+        }
+        int cnt = 0;
+        for (int j = 0; j < nb; ++j)
+            if (keep[j]) {
+                if (cnt >= dm->max_sel) {
+                    #pragma omp atomic write
+                    err = -2;
+                    break;
+                }
+                sel_idx[bh * dm->max_sel + cnt++] = j;
+            }
+        sel_count[bh] = cnt;
+        if (margin) margin[bh] = mg_row;
+        free(keep);
+        free(r);
+    }
+    return err;
+}
+
+/* ---------------------------------------------------------- 5. attention */
+
+/*
+ * out[b][t][i][c] for the (b, h) units listed in `units` (pairs b, h; NULL
+ * means all units): softmax attention of query head i (i / G == h) over
+ * every token of the kept blocks of (b, h) that exists (position < L) and is
+ * not in the future of query token t (query t sits at position L - Tq + t;
+ * the chunk's own keys are already in the cache).  A row with no visible
+ * token is all zeros.
+ */
+int spo_attend(const spo_dims *dm, const spo_params *pr, const uint16_t *q,
+               const void *k_cache, const void *v_cache, const float *k_scale,
+               const float *v_scale, const int32_t *block_table,
+               const int32_t *seq_lens, const int32_t *sel_idx,
+               const int32_t *sel_count, const int32_t *units, int n_units,
+               double *out)
+{
+    const int D = dm->head_dim, H = dm->num_kv_heads, Tq = dm->q_tokens;
+    const int P = dm->block_size, Hq = dm->num_q_heads, G = Hq / H;
+    const double scale = softmax_scale(dm, pr);
+    int total = units ? n_units : dm->batch * H;
+    #pragma omp parallel for schedule(dynamic)
+    for (int u = 0; u < total; ++u) {
+        int b = units ? units[2 * u] : u / H;
+        int h = units ? units[2 * u + 1] : u % H;
+        int L = seq_lens[b];
+        int64_t bh = (int64_t)b * H + h;
+        int cnt = sel_count[bh];
+        int ntok_max = cnt * P;
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(ntok_max > 0 ? ntok_max : 1));
+        int64_t *tpage = (int64_t *)malloc(sizeof(int64_t) * (size_t)(ntok_max > 0 ? ntok_max : 1));
+        int *tslot = (int *)malloc(sizeof(int) * (size_t)(ntok_max > 0 ? ntok_max : 1));
+        for (int t = 0; t < Tq; ++t) {
+            int64_t qpos = (int64_t)L - Tq + t;
+            for (int g = 0; g < G; ++g) {
+                int i = h * G + g;
+                const uint16_t *qr = q + (((int64_t)b * Tq + t) * Hq + i) * D;
+                double *o = out + (((int64_t)b * Tq + t) * Hq + i) * D;
+                int n = 0;
+                for (int s = 0; s < cnt; ++s) {
+                    int j = sel_idx[bh * dm->max_sel + s];
+                    int64_t page = block_table[(int64_t)b * dm->max_blocks + j];
+                    for (int tt = 0; tt < P; ++tt) {
+                        int64_t pos = (int64_t)j * P + tt;
+                        if (pos >= L || pos > qpos)
+                            continue;
+                        double dot = 0.0;
+                        for (int c = 0; c < D; ++c)
+                            dot += spo_bf16_to_f64(qr[c]) *
+                                   cache_at(dm, k_cache, k_scale, page, h, tt, c);
+                        logit[n] = dot * scale;
+                        tpage[n] = page;
+                        tslot[n] = tt;
+                        ++n;
+                    }
+                }
+                for (int c = 0; c < D; ++c)
+                    o[c] = 0.0;
+                if (n == 0)
+                    continue;
+                double mx = logit[0];
+                for (int k = 1; k < n; ++k)
+                    if (logit[k] > mx) mx = logit[k];
+                double z = 0.0;
+                for (int k = 0; k < n; ++k)
+                    z += exp(logit[k] - mx);
+                for (int k = 0; k < n; ++k) {
+                    double p = exp(logit[k] - mx) / z;
+                    for (int c = 0; c < D; ++c)
+                        o[c] += p * cache_at(dm, v_cache, v_scale, tpage[k], h, tslot[k], c);
+                }
+            }
+        }
+        free(logit);
+        free(tpage);
+        free(tslot);
+    }
+    return 0;
+}
+
+/* Threads the OpenMP runtime will use (1 when built without OpenMP). */
+int spo_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
