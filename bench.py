@@ -1,0 +1,428 @@
+"""Benchmark: block-sparse decode attention at 128K context on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload NAME]
+
+One step is one pass of the whole decode path over the workload's batch:
+incremental key compression of each request's tail block, block scores,
+selection (sink + local + top-p/top-k), sparse attention and the split
+merge, all through the C ABI (captured once into CUDA graphs and replayed).
+Inputs are seeded synthetic data resident in HBM; L2 is flushed (a 512 MB
+write) between timed steps, outside the timed events.
+
+Metric: selected-KV HBM GB/s = algorithmic bytes of a step (kept K+V tiles,
+fp8 scales, compressed keys of the scored middle blocks, q, out) / step time,
+aggregated over ranks; decode queries/s alongside.  Under torchrun each rank
+runs its own independent batch (weak scaling, no collective on the data
+path); the step time is the max over ranks.
+
+--impl reference times the float64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_kv_spattn_b200.workloads import BENCH_WORKLOAD, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "selected-KV HBM GB/s (% of ~8 TB/s) and decode queries/s at 128K ctx, 1 B200"
+FLUSH_BYTES = 512 << 20
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
+ATTN_SOURCES = ["common.cuh", "attention.cuh"]
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "block_sparse_kv_spattn_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(units_in_launch: float):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    capture, scaled to this launch; None if the kernel changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("source_sha") != attn_source_hash():
+        return None
+    return t["dram_bytes_per_launch"] * units_in_launch / t["units_per_launch"]
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        rows = []
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                rows.append((float(f[0]), float(f[1]), f[3:7]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def step_bytes(inp, sel_count: torch.Tensor) -> dict:
+    """Algorithmic bytes of one step (one rank)."""
+    w = inp["workload"]
+    P, D, H = w.block_size, w.head_dim, w.num_kv_heads
+    elt = 1 if w.kv_fp8 else 2
+    kept = int(sel_count.sum())
+    kv = kept * P * D * elt * 2 + (kept * 8 if w.kv_fp8 else 0)
+    n_mid = sum(max(0, (int(L) + P - 1) // P - w.sink_blocks - w.local_blocks)
+                for L in inp["seq_lens"].tolist())
+    kbar = n_mid * H * D * 4
+    q = inp["q"].numel() * 2
+    out = inp["q"].numel() * 4
+    return dict(kv=kv, kbar=kbar, q=q, out=out, total=kv + kbar + q + out, kept_block_heads=kept)
+
+
+def run_native(args, rank, world, local_rank):
+    from block_sparse_kv_spattn_b200 import spattn
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    q, kc, vc, ks, vs = inp["q"], inp["k_cache"], inp["v_cache"], inp["k_scale"], inp["v_scale"]
+    bt, sl = inp["block_table"], inp["seq_lens"]
+    params = spattn.Params(sink_blocks=w.sink_blocks, local_blocks=w.local_blocks, mode=w.mode,
+                           top_k=w.top_k, top_p=w.top_p, max_ratio=w.max_ratio)
+    dims = spattn.dims_for(q, kc, bt)
+    max_sel = spattn.required_max_sel(dims, params)
+    dims.max_sel = max_sel
+    B, Tq, Hkv = w.batch, w.q_tokens, w.num_kv_heads
+    kbar = torch.empty((kc.shape[0], Hkv, w.head_dim), dtype=torch.float32, device=dev)
+    spattn.compress_keys(kc, ks, bt, sl, kbar, num_q_heads=w.num_q_heads, q_tokens=Tq)
+    old_lens = (sl - Tq).clamp_min(0).to(torch.int32)
+    scores = torch.empty((B, Tq, Hkv, bt.shape[1]), dtype=torch.float32, device=dev)
+    sel_idx = torch.empty((B, Hkv, max_sel), dtype=torch.int32, device=dev)
+    sel_count = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+    out = torch.empty(tuple(q.shape), dtype=torch.float32, device=dev)
+    ws = spattn.alloc_workspace(dims, params, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def front():   # append-side compression of the tail block, scores, selection
+        spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
+                             q_tokens=Tq)
+        spattn.block_scores(q, kbar, bt, sl, scores, params, k_cache=kc)
+        spattn.select(scores, sl, sel_idx, sel_count, params, q=q, k_cache=kc, block_table=bt)
+
+    def attend():  # sparse attention + split merge
+        spattn.decode_selected(q, kc, vc, ks, vs, bt, sl, sel_idx, sel_count, out, ws, params)
+
+    # warm up eagerly once (sets kernel attributes), then capture graphs
+    front()
+    attend()
+    torch.cuda.synchronize()
+    status = spattn.device_status()
+    if status:
+        raise RuntimeError(f"device status {status:#x}")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        g_front, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_front, stream=s):
+            front()
+        with torch.cuda.graph(g_attn, stream=s):
+            attend()
+    torch.cuda.current_stream().wait_stream(s)
+    launches_per_step = 5          # compress, scores, select, attention, merge
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        g_front.replay()
+        g_attn.replay()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    smi_id = (f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+              if hasattr(props, "pci_bus_id") else str(local_rank))
+    with Clocks(smi_id) as clk:
+        t_wall = time.perf_counter()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record()
+            g_front.replay()
+            ev[i][1].record()
+            g_attn.replay()
+            ev[i][2].record()
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(step_ms)
+    bts = step_bytes(inp, sel_count)
+    status = spattn.device_status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} after the timed region")
+
+    # e2e: q / seq_lens in from pinned host memory, out back, every step
+    q_h = q.cpu().pin_memory()
+    sl_h = sl.cpu().pin_memory()
+    out_h = torch.empty(tuple(out.shape), dtype=out.dtype).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        e2e_ev[i][0].record()
+        q.copy_(q_h, non_blocking=True)
+        sl.copy_(sl_h, non_blocking=True)
+        g_front.replay()
+        g_attn.replay()
+        out_h.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev)
+
+    t = torch.tensor([total_ms, sum(attn_ms), e2e_ms, float(bts["total"]), float(bts["kv"] + bts["q"] + bts["out"])],
+                     dtype=torch.float64, device=dev)
+    if world > 1:
+        mx = t[:3].clone()
+        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
+        sm = t[3:].clone()
+        torch.distributed.all_reduce(sm, op=torch.distributed.ReduceOp.SUM)
+        t = torch.cat([mx, sm])
+    total_ms, attn_total_ms, e2e_total_ms, all_bytes, _ = t.tolist()
+    if rank != 0:
+        return None
+    ms_per_step = total_ms / K
+    value = all_bytes / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    attn_ms_mean = attn_total_ms / K
+    attn_bytes = bts["kv"] + bts["q"] + bts["out"]     # one rank's launch
+    achieved = attn_bytes / (attn_ms_mean * 1e-3) / 1e9
+    traffic = measured_traffic(bts["kept_block_heads"])
+    queries = B * Tq * world / (ms_per_step * 1e-3)
+    e2e_value = all_bytes / (e2e_total_ms / K * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8" if w.kv_fp8 else "bf16",
+        "data": "synthetic (seeded; power-law block importance)",
+        "config": {"workload": w.name, "batch": B, "q_tokens": Tq, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": Hkv, "seq_len": w.seq_len, "block": w.block_size,
+                   "sink_blocks": w.sink_blocks, "local_blocks": w.local_blocks,
+                   "selection": f"{w.mode} p={w.top_p} cap={w.max_ratio}" if w.mode == "topp" else
+                   f"{w.mode} k={w.top_k} ratio={w.max_ratio}",
+                   "l2": "flushed between steps (512 MB write, outside the timed events)",
+                   "parallelism": f"independent replicas x{world}"},
+        "hbm_fraction": round(value / peak, 4),
+        "queries_per_s": round(queries, 1),
+        "bytes_per_step": bts,
+        "roofline": {"kernel": "attention (attn_kernel + merge_kernel, one decode_selected call)",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": None if traffic is None else int(traffic),
+                     "ms_per_launch": round(attn_ms_mean, 5)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": q.numel() * 2 + sl.numel() * 4,
+                "d2h_bytes_per_step": out.numel() * 4},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk.summary(),
+        "wall_s": round(t_wall, 3),
+    }
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(inp, bts, ms_per_step)
+    return line
+
+
+def cpu_baseline(inp, bts, gpu_ms):
+    """The float64 oracle on this host's cores, on a bounded sample: all KV
+    heads of request 0 (scores, selection, attention; compressed keys are
+    computed outside the timing), scaled to the whole step."""
+    import oracle
+    from tests.oracle_io import bits16, cache_bytes, dims_of, params_of
+    from tests.parity import subproblem
+
+    w = inp["workload"]
+    sub = subproblem(inp, 0)
+    dims = dims_of(sub)
+    par = params_of(w)
+    qh, kh, vh = bits16(sub["q"]), cache_bytes(sub["k_cache"]), cache_bytes(sub["v_cache"])
+    ksc, vsc = sub["k_scale"].cpu().numpy(), sub["v_scale"].cpu().numpy()
+    bt, sl = sub["block_table"].cpu().numpy(), sub["seq_lens"].cpu().numpy()
+    kbar = oracle.compress_keys(dims, kh, ksc, bt, sl)
+    times = []
+    t_end = time.perf_counter() + 10.0
+    while time.perf_counter() < t_end or not times:
+        t0 = time.perf_counter()
+        sc = oracle.block_scores(dims, par, qh, kbar, bt, sl)
+        sel, cnt, _ = oracle.select(dims, par, sc, sl)
+        oracle.attend(dims, par, qh, kh, vh, ksc, vsc, bt, sl, sel, cnt)
+        times.append(time.perf_counter() - t0)
+    per_req = statistics.median(times)
+    step_s = per_req * w.batch
+    return {"value": round(bts["total"] / step_s / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"request 0 of {w.batch} (all {w.num_kv_heads} KV heads), {len(times)} runs, "
+                      f"median {per_req:.3f} s, scaled x{w.batch} to the step",
+            "ms_per_step": round(step_s * 1e3, 3), "gpu_speedup": round(step_s * 1e3 / gpu_ms, 1)}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: rank 0 only, bounded per-step sample."""
+    if rank != 0:
+        return None
+    import oracle
+    from tests.oracle_io import bits16, cache_bytes, dims_of, params_of
+    from tests.parity import subproblem
+
+    w = WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(w, device=dev)
+    par = params_of(w)
+    subs = []
+    # per step: one (request, KV head) unit of the workload, cycling
+    for b in range(min(w.batch, 2)):
+        sub = subproblem(inp, b)
+        dims = dims_of(sub)
+        qh, kh, vh = bits16(sub["q"]), cache_bytes(sub["k_cache"]), cache_bytes(sub["v_cache"])
+        ksc, vsc = sub["k_scale"].cpu().numpy(), sub["v_scale"].cpu().numpy()
+        bt, sl = sub["block_table"].cpu().numpy(), sub["seq_lens"].cpu().numpy()
+        kbar = oracle.compress_keys(dims, kh, ksc, bt, sl)
+        subs.append((dims, qh, kh, vh, ksc, vsc, bt, sl, kbar))
+    units = w.batch * w.num_kv_heads
+
+    def one(i):
+        dims, qh, kh, vh, ksc, vsc, bt, sl, kbar = subs[i % len(subs)]
+        h = (i // len(subs)) % w.num_kv_heads
+        sc = oracle.block_scores(dims, par, qh, kbar, bt, sl)
+        sel, cnt, _ = oracle.select(dims, par, sc, sl)
+        oracle.attend(dims, par, qh, kh, vh, ksc, vsc, bt, sl, sel, cnt, units=[(0, h)])
+        return int(cnt[0, h])
+
+    for i in range(args.warmup):
+        one(i)
+    times, kept = [], 0
+    budget = time.perf_counter() + 150.0
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        kept += one(i)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() > budget:
+            break
+    per_unit = statistics.mean(times)
+    step_s = per_unit * units
+    # bytes of a full step at the sampled units' mean kept count
+    P, D = w.block_size, w.head_dim
+    elt = 1 if w.kv_fp8 else 2
+    mean_kept = kept / len(times)
+    nbs = [(int(L) + P - 1) // P for L in inp["seq_lens"].tolist()]
+    n_mid = sum(max(0, nb - w.sink_blocks - w.local_blocks) for nb in nbs)
+    total = units * mean_kept * P * D * elt * 2 + n_mid * w.num_kv_heads * D * 4 + inp["q"].numel() * 6
+    value = total / step_s / 1e9
+    sample = (f"{len(times)} steps x one (request, KV head) unit of {units} (scores, selection, attention "
+              f"in float64), scaled x{units} to the step")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
+        "n_gpus": world, "steps": len(times), "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; power-law block importance)",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "native":
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_native(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

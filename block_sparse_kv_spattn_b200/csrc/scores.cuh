@@ -1,0 +1,145 @@
+// scores.cuh -- score every middle block against its compressed key.
+//
+// "CSA + HCA 混合注意力机制" §4.2 (Lightning Indexer, steps 3-4: every
+// compressed entry gets a score from the query, heads are aggregated into one
+// score per entry) and §4.4 step 1.  Without learned indexer projections the
+// score of block j for KV head h is the mean of the group's per-head logits
+// against the block's mean key: (qbar . kbar_j) * sm_scale, qbar the mean of
+// the group's query rows.
+#pragma once
+
+#include "common.cuh"
+
+namespace spattn {
+
+struct ScoresArgs {
+    const uint16_t *q;        // bf16 bits [B][Tq][Hq][D]
+    const float *kbar;        // [num_pages][Hkv][D]
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    float *scores;            // [B][Tq][Hkv][max_blocks]
+    int tq, hq, num_pages, max_blocks, sink, local;
+    float scale;
+};
+
+constexpr int kScoreThreads = 256;
+constexpr int kScoreBlocksPerCta = 64;
+
+// Sum of v[0..7] over the 32 lanes, scattered: afterwards lane l holds the
+// full sum of element (l >> 2) & 7 in v[0].  Butterfly halving at offsets 16,
+// 8, 4 (each lane keeps the half named by its offset bit), then plain xor
+// reductions at 2 and 1: 9 shuffles for 8 warp sums.
+__device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int step = 0; step < 3; ++step) {
+        const int off = 16 >> step;
+        const int half = 4 >> step;
+        const bool up = lane & off;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            float send = up ? v[i] : v[i + half];
+            float keep = up ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    float r = v[0];
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    return r;
+}
+
+// Grid (ceil(max_blocks / 64), B).  Dynamic shared memory:
+// qbar [Tq][HKV][D] fp32 followed by a [Tq*HKV][64] fp32 output tile.
+template <int HKV>
+__global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs a) {
+    extern __shared__ float4 smem_f4[];
+    float *qbar = reinterpret_cast<float *>(smem_f4);
+    float *tile = qbar + a.tq * HKV * kHeadDim;
+    const int b = blockIdx.y;
+    const int j0 = blockIdx.x * kScoreBlocksPerCta;
+    const int G = a.hq / HKV;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int rows = a.tq * HKV;
+
+    int L = a.seq_lens[b];
+    if (L < 0 || L > a.max_blocks * kBlock) {
+        if (threadIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
+        L = 0;
+    }
+    const int nb = (L + kBlock - 1) / kBlock;
+
+    // 1. group-mean query rows
+    for (int idx = threadIdx.x; idx < rows * kHeadDim; idx += kScoreThreads) {
+        const int c = idx % kHeadDim, th = idx / kHeadDim;
+        const int hh = th % HKV, t = th / HKV;
+        const uint16_t *qr = a.q + (((int64_t)b * a.tq + t) * a.hq + hh * G) * kHeadDim + c;
+        float s = 0.f;
+        for (int g = 0; g < G; ++g) s += __uint_as_float((uint32_t)qr[g * kHeadDim] << 16);
+        qbar[idx] = s / (float)G;
+    }
+    __syncthreads();
+
+    // 2. one warp per block j; lane owns columns [4*lane, 4*lane+4)
+    constexpr int HPC = HKV < 8 ? HKV : 8;      // heads per 8-value chunk
+    constexpr int TPC = 8 / HPC;                // tokens per chunk
+    for (int jj = warp; jj < kScoreBlocksPerCta; jj += kScoreThreads / 32) {
+        const int j = j0 + jj;
+        if (j >= a.max_blocks) break;
+        const bool middle = j >= a.sink && j < nb - a.local;
+        if (!middle) {
+            for (int r = lane; r < rows; r += 32) tile[r * kScoreBlocksPerCta + jj] = -INFINITY;
+            continue;
+        }
+        const int page = a.block_table[(int64_t)b * a.max_blocks + j];
+        if (page < 0 || page >= a.num_pages) {
+            if (lane == 0) flag(SPATTN_DEV_BAD_PAGE);
+            for (int r = lane; r < rows; r += 32) tile[r * kScoreBlocksPerCta + jj] = -INFINITY;
+            continue;
+        }
+        float4 kv[HKV];
+        const float4 *kp = reinterpret_cast<const float4 *>(a.kbar + (int64_t)page * HKV * kHeadDim);
+#pragma unroll
+        for (int hh = 0; hh < HKV; ++hh) kv[hh] = kp[hh * (kHeadDim / 4) + lane];
+
+        for (int t0 = 0; t0 < a.tq; t0 += TPC) {
+#pragma unroll
+            for (int h0 = 0; h0 < HKV; h0 += HPC) {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int tt = t0 + i / HPC, hh = h0 + i % HPC;
+                    float s = 0.f;
+                    if (tt < a.tq) {
+                        const float4 qv =
+                            reinterpret_cast<const float4 *>(qbar + (tt * HKV + hh) * kHeadDim)[lane];
+                        s = qv.x * kv[hh].x;
+                        s = fmaf(qv.y, kv[hh].y, s);
+                        s = fmaf(qv.z, kv[hh].z, s);
+                        s = fmaf(qv.w, kv[hh].w, s);
+                    }
+                    v[i] = s;
+                }
+                const float r = reduce_scatter8(v);
+                if ((lane & 3) == 0) {
+                    const int i = lane >> 2;
+                    const int tt = t0 + i / HPC, hh = h0 + i % HPC;
+                    if (tt < a.tq) tile[(tt * HKV + hh) * kScoreBlocksPerCta + jj] = r * a.scale;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // 3. coalesced store of the tile
+    for (int idx = threadIdx.x; idx < rows * kScoreBlocksPerCta; idx += kScoreThreads) {
+        const int jj = idx % kScoreBlocksPerCta, r = idx / kScoreBlocksPerCta;
+        const int j = j0 + jj;
+        if (j < a.max_blocks) {
+            const int hh = r % HKV, t = r / HKV;
+            a.scores[(((int64_t)b * a.tq + t) * HKV + hh) * a.max_blocks + j] = tile[idx];
+        }
+    }
+}
+
+}  // namespace spattn

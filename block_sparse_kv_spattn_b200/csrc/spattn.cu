@@ -1,0 +1,515 @@
+// spattn.cu -- C ABI of libspattn: argument checks, workspace layout and
+// kernel launches.  Every kernel lives in the headers included below; this
+// is the only translation unit, so the device status word is one symbol.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <set>
+#include <string>
+#include <utility>
+
+#include "spattn.h"
+#include "common.cuh"
+#include "compress.cuh"
+#include "scores.cuh"
+#include "select.cuh"
+#include "attention.cuh"
+
+using namespace spattn;
+
+namespace {
+
+thread_local std::string g_err;
+
+spattn_status fail(spattn_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+spattn_status ok() {
+    g_err.clear();
+    return SPATTN_OK;
+}
+
+#define SP_TRY(expr)                                  \
+    do {                                              \
+        spattn_status _st = (expr);                   \
+        if (_st != SPATTN_OK) return _st;             \
+    } while (0)
+
+spattn_status cuda_ok(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return SPATTN_OK;
+    return fail(SPATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Upper bound on persistent attention CTAs (2 per SM); the workspace is sized
+// for it so that workspace sizes need no device query.
+constexpr int kMaxAttnCtas = 2 * 160;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool pow2_hkv(int h) { return h == 1 || h == 2 || h == 4 || h == 8 || h == 16; }
+
+spattn_status check_dims(const spattn_dims *d) {
+    if (!d) return fail(SPATTN_ERR_INVALID_ARG, "dims is NULL");
+    if (d->batch < 1 || d->q_tokens < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1 ||
+        d->num_pages < 1 || d->max_blocks_per_seq < 1 || d->max_sel < 0)
+        return fail(SPATTN_ERR_INVALID_ARG, "dims: sizes must be positive");
+    if (d->head_dim != kHeadDim)
+        return fail(SPATTN_ERR_UNSUPPORTED, "head_dim %d: only %d is built", d->head_dim, kHeadDim);
+    if (d->block_size != kBlock)
+        return fail(SPATTN_ERR_UNSUPPORTED, "block_size %d: only %d is built", d->block_size, kBlock);
+    if (d->num_q_heads % d->num_kv_heads)
+        return fail(SPATTN_ERR_INVALID_ARG, "num_q_heads %d is not a multiple of num_kv_heads %d",
+                    d->num_q_heads, d->num_kv_heads);
+    if (!pow2_hkv(d->num_kv_heads))
+        return fail(SPATTN_ERR_UNSUPPORTED, "num_kv_heads %d: built for 1, 2, 4, 8, 16", d->num_kv_heads);
+    const int64_t rows = (int64_t)d->q_tokens * (d->num_q_heads / d->num_kv_heads);
+    if (rows > 64)
+        return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_q_heads / num_kv_heads = %lld > 64",
+                    (long long)rows);
+    if (d->kv_dtype != SPATTN_KV_BF16 && d->kv_dtype != SPATTN_KV_FP8_E4M3)
+        return fail(SPATTN_ERR_INVALID_ARG, "kv_dtype %d", d->kv_dtype);
+    if ((int64_t)d->max_blocks_per_seq * kBlock > INT32_MAX / 2)
+        return fail(SPATTN_ERR_UNSUPPORTED, "max_blocks_per_seq too large");
+    return SPATTN_OK;
+}
+
+spattn_status check_params(const spattn_params *p) {
+    if (!p) return fail(SPATTN_ERR_INVALID_ARG, "params is NULL");
+    if (p->sink_blocks < 0 || p->local_blocks < 0)
+        return fail(SPATTN_ERR_INVALID_ARG, "sink_blocks and local_blocks must be >= 0");
+    if (p->mode != SPATTN_SEL_TOPK && p->mode != SPATTN_SEL_TOPP)
+        return fail(SPATTN_ERR_INVALID_ARG, "mode %d", p->mode);
+    if (p->top_k < 0) return fail(SPATTN_ERR_INVALID_ARG, "top_k %d < 0", p->top_k);
+    if (p->mode == SPATTN_SEL_TOPP && !(p->top_p > 0.f && p->top_p <= 1.f))
+        return fail(SPATTN_ERR_INVALID_ARG, "top_p %g not in (0, 1]", (double)p->top_p);
+    if (!(p->max_ratio >= 0.f && p->max_ratio <= 1.f))
+        return fail(SPATTN_ERR_INVALID_ARG, "max_ratio %g not in [0, 1]", (double)p->max_ratio);
+    if (!(p->sm_scale >= 0.f) || !std::isfinite(p->sm_scale))
+        return fail(SPATTN_ERR_INVALID_ARG, "sm_scale %g", (double)p->sm_scale);
+    return SPATTN_OK;
+}
+
+int n_mid_cap(const spattn_dims *d, const spattn_params *p) {
+    const int64_t n = (int64_t)d->max_blocks_per_seq - p->sink_blocks - p->local_blocks;
+    return n > 0 ? (int)n : 0;
+}
+
+int k_max_of(const spattn_params *p, int n_mid) {
+    if (p->max_ratio > 0.f) {
+        const int k = (int)std::floor((double)p->max_ratio * (double)n_mid);
+        return k < n_mid ? k : n_mid;
+    }
+    return n_mid;
+}
+
+int32_t required_max_sel(const spattn_dims *d, const spattn_params *p) {
+    const int nm = n_mid_cap(d, p);
+    const int km = k_max_of(p, nm);
+    int k = km;
+    if (p->mode == SPATTN_SEL_TOPK && p->top_k > 0 && p->top_k < k) k = p->top_k;
+    const int64_t mid = std::min<int64_t>(nm, (int64_t)d->q_tokens * k);
+    const int64_t req = (int64_t)p->sink_blocks + p->local_blocks + mid;
+    return (int32_t)std::min<int64_t>(req, d->max_blocks_per_seq);
+}
+
+float sm_scale_of(const spattn_params *p) {
+    return p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt((float)kHeadDim);
+}
+
+int rows_of(const spattn_dims *d) { return d->q_tokens * (d->num_q_heads / d->num_kv_heads); }
+
+int rg_of(int rows) {
+    const int rg = (rows + 3) / 4;
+    int p = 1;
+    while (p < rg) p <<= 1;
+    return p;
+}
+
+// Per-device caches (SM count; which kernels have their shared-memory limit
+// raised).  Guarded by one mutex: these are host-side set-up calls only.
+std::mutex g_mu;
+std::set<std::pair<int, const void *>> g_smem_set;
+
+spattn_status ensure_smem(const void *func, int bytes) {
+    if (bytes <= 48 * 1024) return SPATTN_OK;
+    int dev;
+    SP_TRY(cuda_ok(cudaGetDevice(&dev), "cudaGetDevice"));
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_smem_set.count({dev, func})) return SPATTN_OK;
+    SP_TRY(cuda_ok(cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+                   "cudaFuncSetAttribute"));
+    g_smem_set.insert({dev, func});
+    return SPATTN_OK;
+}
+
+std::map<int, int> g_sms;
+
+// SM count of the current device, queried once per device (so that calls
+// captured into a CUDA graph after the first one make no attribute query).
+spattn_status sm_count(int *out) {
+    int dev;
+    SP_TRY(cuda_ok(cudaGetDevice(&dev), "cudaGetDevice"));
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_sms.find(dev);
+    if (it != g_sms.end()) {
+        *out = it->second;
+        return SPATTN_OK;
+    }
+    SP_TRY(cuda_ok(cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev),
+                   "cudaDeviceGetAttribute"));
+    g_sms[dev] = *out;
+    return SPATTN_OK;
+}
+
+constexpr int kMaxSmem = 227 * 1024;
+
+struct DecodeLayout {
+    size_t scores_off, scores_bytes, part_o_off, part_ml_off, total;
+};
+
+DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
+    DecodeLayout L{};
+    const int64_t units = (int64_t)d->batch * d->num_kv_heads;
+    const int64_t slots = kMaxAttnCtas + units;
+    const int rows = rows_of(d);
+    size_t off = 0;
+    L.scores_off = 0;
+    L.scores_bytes = with_scores ? align_up((size_t)d->batch * d->q_tokens * d->num_kv_heads *
+                                            d->max_blocks_per_seq * sizeof(float))
+                                 : 0;
+    off += L.scores_bytes;
+    L.part_o_off = off;
+    off += align_up((size_t)slots * rows * kHeadDim * sizeof(float));
+    L.part_ml_off = off;
+    off += align_up((size_t)slots * rows * 2 * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------- launches
+
+spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const void *q,
+                            const float *kbar, const int32_t *bt, const int32_t *sl, float *scores,
+                            cudaStream_t st) {
+    ScoresArgs a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.kbar = kbar;
+    a.block_table = bt;
+    a.seq_lens = sl;
+    a.scores = scores;
+    a.tq = d->q_tokens;
+    a.hq = d->num_q_heads;
+    a.num_pages = d->num_pages;
+    a.max_blocks = d->max_blocks_per_seq;
+    a.sink = p->sink_blocks;
+    a.local = p->local_blocks;
+    a.scale = sm_scale_of(p);
+    const int rowsq = d->q_tokens * d->num_kv_heads;
+    const int smem = rowsq * (kHeadDim + kScoreBlocksPerCta) * (int)sizeof(float);
+    if (smem > kMaxSmem)
+        return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_kv_heads = %d too large for block scores", rowsq);
+    dim3 grid((d->max_blocks_per_seq + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta, d->batch);
+    const void *fn = nullptr;
+    switch (d->num_kv_heads) {
+        case 1: fn = (const void *)block_scores_kernel<1>; break;
+        case 2: fn = (const void *)block_scores_kernel<2>; break;
+        case 4: fn = (const void *)block_scores_kernel<4>; break;
+        case 8: fn = (const void *)block_scores_kernel<8>; break;
+        case 16: fn = (const void *)block_scores_kernel<16>; break;
+    }
+    SP_TRY(ensure_smem(fn, smem));
+    switch (d->num_kv_heads) {
+        case 1: block_scores_kernel<1><<<grid, kScoreThreads, smem, st>>>(a); break;
+        case 2: block_scores_kernel<2><<<grid, kScoreThreads, smem, st>>>(a); break;
+        case 4: block_scores_kernel<4><<<grid, kScoreThreads, smem, st>>>(a); break;
+        case 8: block_scores_kernel<8><<<grid, kScoreThreads, smem, st>>>(a); break;
+        case 16: block_scores_kernel<16><<<grid, kScoreThreads, smem, st>>>(a); break;
+    }
+    return cuda_ok(cudaGetLastError(), "block_scores launch");
+}
+
+spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const float *scores,
+                            const int32_t *sl, int32_t *sel_idx, int32_t *sel_count, cudaStream_t st) {
+    SelectArgs a;
+    a.scores = scores;
+    a.seq_lens = sl;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.tq = d->q_tokens;
+    a.hkv = d->num_kv_heads;
+    a.max_blocks = d->max_blocks_per_seq;
+    a.max_sel = d->max_sel;
+    a.sink = p->sink_blocks;
+    a.local = p->local_blocks;
+    a.mode = p->mode;
+    a.top_k = p->top_k;
+    a.top_p = p->top_p;
+    a.max_ratio = p->max_ratio;
+    a.n_mid_cap = std::max(1, n_mid_cap(d, p));
+    a.sort_cap = 0;
+    if (p->mode == SPATTN_SEL_TOPP) {
+        const int km = std::max(1, k_max_of(p, n_mid_cap(d, p)));
+        int np2 = 1;
+        while (np2 < km) np2 <<= 1;
+        a.sort_cap = np2;
+    }
+    const size_t smem = select_smem_bytes(a.n_mid_cap, a.sort_cap, a.max_blocks);
+    if (smem > (size_t)kMaxSmem)
+        return fail(SPATTN_ERR_UNSUPPORTED, "selection needs %zu bytes of shared memory (max_blocks %d)",
+                    smem, a.max_blocks);
+    SP_TRY(ensure_smem((const void *)select_kernel, (int)smem));
+    select_kernel<<<d->batch * d->num_kv_heads, kSelThreads, smem, st>>>(a);
+    return cuda_ok(cudaGetLastError(), "select launch");
+}
+
+template <int RG, bool FP8>
+spattn_status launch_attn_t(const AttnArgs &a, int ctas, cudaStream_t st) {
+    const int smem = attn_smem_bytes(FP8, RG);
+    SP_TRY(ensure_smem((const void *)attn_kernel<RG, FP8>, smem));
+    attn_kernel<RG, FP8><<<ctas, kAttnThreads, smem, st>>>(a);
+    return cuda_ok(cudaGetLastError(), "attention launch");
+}
+
+template <bool FP8>
+spattn_status launch_attn_rg(int rg, const AttnArgs &a, int ctas, cudaStream_t st) {
+    switch (rg) {
+        case 1: return launch_attn_t<1, FP8>(a, ctas, st);
+        case 2: return launch_attn_t<2, FP8>(a, ctas, st);
+        case 4: return launch_attn_t<4, FP8>(a, ctas, st);
+        case 8: return launch_attn_t<8, FP8>(a, ctas, st);
+        case 16: return launch_attn_t<16, FP8>(a, ctas, st);
+    }
+    return fail(SPATTN_ERR_UNSUPPORTED, "row groups %d", rg);
+}
+
+spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, const void *q,
+                               const void *k_cache, const void *v_cache, const float *k_scale,
+                               const float *v_scale, const int32_t *bt, const int32_t *sl,
+                               const int32_t *sel_idx, const int32_t *sel_count, float *out,
+                               float *part_o, float *part_ml, cudaStream_t st) {
+    const bool fp8 = d->kv_dtype == SPATTN_KV_FP8_E4M3;
+    const int rows = rows_of(d);
+    const int rg = rg_of(rows);
+    int sms;
+    SP_TRY(sm_count(&sms));
+    const int per_sm = rg > 8 ? 1 : 2;
+    const int ctas = std::min(kMaxAttnCtas, sms * per_sm);
+    AttnArgs a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.k_cache = static_cast<const uint8_t *>(k_cache);
+    a.v_cache = static_cast<const uint8_t *>(v_cache);
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.block_table = bt;
+    a.seq_lens = sl;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.part_o = part_o;
+    a.part_ml = part_ml;
+    a.tq = d->q_tokens;
+    a.hq = d->num_q_heads;
+    a.hkv = d->num_kv_heads;
+    a.group = d->num_q_heads / d->num_kv_heads;
+    a.rows = rows;
+    a.units = d->batch * d->num_kv_heads;
+    a.num_pages = d->num_pages;
+    a.max_blocks = d->max_blocks_per_seq;
+    a.max_sel = d->max_sel;
+    a.qscale = sm_scale_of(p) * kLog2e;
+    SP_TRY(fp8 ? launch_attn_rg<true>(rg, a, ctas, st) : launch_attn_rg<false>(rg, a, ctas, st));
+
+    MergeArgs m;
+    m.part_o = part_o;
+    m.part_ml = part_ml;
+    m.sel_count = sel_count;
+    m.out = out;
+    m.batch = d->batch;
+    m.tq = d->q_tokens;
+    m.hq = d->num_q_heads;
+    m.hkv = d->num_kv_heads;
+    m.group = a.group;
+    m.rows = rows;
+    m.units = a.units;
+    m.max_sel = d->max_sel;
+    m.ctas = ctas;
+    const int64_t nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
+    const int per = kMergeThreads / 32;
+    merge_kernel<<<(unsigned)((nrows + per - 1) / per), kMergeThreads, 0, st>>>(m);
+    return cuda_ok(cudaGetLastError(), "merge launch");
+}
+
+spattn_status check_cache_args(const spattn_dims *d, const void *q, const void *k_cache,
+                               const void *v_cache, const float *k_scale, const float *v_scale,
+                               const int32_t *bt, const int32_t *sl) {
+    if (!q || !k_cache || !v_cache || !bt || !sl)
+        return fail(SPATTN_ERR_INVALID_ARG, "q, k_cache, v_cache, block_table, seq_lens are required");
+    if (d->kv_dtype == SPATTN_KV_FP8_E4M3 && (!k_scale || !v_scale))
+        return fail(SPATTN_ERR_INVALID_ARG, "fp8 caches need k_scale and v_scale");
+    if (((uintptr_t)k_cache | (uintptr_t)v_cache) & 15)
+        return fail(SPATTN_ERR_INVALID_ARG, "k_cache and v_cache must be 16-byte aligned");
+    if ((uintptr_t)q & 15) return fail(SPATTN_ERR_INVALID_ARG, "q must be 16-byte aligned");
+    return SPATTN_OK;
+}
+
+}  // namespace
+
+// ================================================================ C ABI
+
+extern "C" {
+
+int32_t spattn_required_max_sel(const spattn_dims *dims, const spattn_params *params) {
+    if (check_dims(dims) != SPATTN_OK || check_params(params) != SPATTN_OK) return -1;
+    return required_max_sel(dims, params);
+}
+
+spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache, const float *k_scale,
+                                   const int32_t *block_table, const int32_t *old_lens,
+                                   const int32_t *seq_lens, float *kbar, spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    if (!k_cache || !block_table || !seq_lens || !kbar)
+        return fail(SPATTN_ERR_INVALID_ARG, "k_cache, block_table, seq_lens, kbar are required");
+    const bool fp8 = dims->kv_dtype == SPATTN_KV_FP8_E4M3;
+    if (fp8 && !k_scale) return fail(SPATTN_ERR_INVALID_ARG, "fp8 caches need k_scale");
+    if (((uintptr_t)k_cache & 15) || ((uintptr_t)kbar & 15))
+        return fail(SPATTN_ERR_INVALID_ARG, "k_cache and kbar must be 16-byte aligned");
+    CompressArgs a;
+    a.k_cache = static_cast<const uint8_t *>(k_cache);
+    a.k_scale = k_scale;
+    a.block_table = block_table;
+    a.old_lens = old_lens;
+    a.seq_lens = seq_lens;
+    a.kbar = kbar;
+    a.hkv = dims->num_kv_heads;
+    a.num_pages = dims->num_pages;
+    a.max_blocks = dims->max_blocks_per_seq;
+    const int gx = old_lens ? (dims->q_tokens + kBlock - 1) / kBlock + 1 : dims->max_blocks_per_seq;
+    dim3 grid(gx, dims->batch);
+    const int threads = dims->num_kv_heads * 16;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (fp8)
+        compress_keys_kernel<true><<<grid, threads, 0, st>>>(a);
+    else
+        compress_keys_kernel<false><<<grid, threads, 0, st>>>(a);
+    SP_TRY(cuda_ok(cudaGetLastError(), "compress_keys launch"));
+    return ok();
+}
+
+spattn_status spattn_block_scores(const spattn_dims *dims, const spattn_params *params, const void *q,
+                                  const float *kbar, const int32_t *block_table,
+                                  const int32_t *seq_lens, float *scores, spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    SP_TRY(check_params(params));
+    if (!q || !kbar || !block_table || !seq_lens || !scores)
+        return fail(SPATTN_ERR_INVALID_ARG, "q, kbar, block_table, seq_lens, scores are required");
+    if (((uintptr_t)kbar & 15)) return fail(SPATTN_ERR_INVALID_ARG, "kbar must be 16-byte aligned");
+    SP_TRY(launch_scores(dims, params, q, kbar, block_table, seq_lens, scores,
+                         reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+spattn_status spattn_select(const spattn_dims *dims, const spattn_params *params, const float *scores,
+                            const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_count,
+                            spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    SP_TRY(check_params(params));
+    if (!scores || !seq_lens || !sel_idx || !sel_count)
+        return fail(SPATTN_ERR_INVALID_ARG, "scores, seq_lens, sel_idx, sel_count are required");
+    const int32_t need = required_max_sel(dims, params);
+    if (dims->max_sel < need)
+        return fail(SPATTN_ERR_INVALID_ARG, "max_sel %d < required %d", dims->max_sel, need);
+    SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count,
+                         reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+size_t spattn_decode_workspace_size(const spattn_dims *dims, const spattn_params *params) {
+    if (check_dims(dims) != SPATTN_OK || check_params(params) != SPATTN_OK) return 0;
+    return decode_layout(dims, true).total;
+}
+
+spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_params *params, const void *q,
+                                     const void *k_cache, const void *v_cache, const float *k_scale,
+                                     const float *v_scale, const int32_t *block_table,
+                                     const int32_t *seq_lens, const int32_t *sel_idx,
+                                     const int32_t *sel_count, float *out, void *workspace,
+                                     size_t workspace_bytes, spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    SP_TRY(check_params(params));
+    SP_TRY(check_cache_args(dims, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens));
+    if (!sel_idx || !sel_count || !out)
+        return fail(SPATTN_ERR_INVALID_ARG, "sel_idx, sel_count, out are required");
+    if ((uintptr_t)out & 15) return fail(SPATTN_ERR_INVALID_ARG, "out must be 16-byte aligned");
+    const DecodeLayout L = decode_layout(dims, false);
+    if (!workspace || workspace_bytes < L.total)
+        return fail(SPATTN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", workspace_bytes, L.total);
+    if ((uintptr_t)workspace & (kAlign - 1))
+        return fail(SPATTN_ERR_WORKSPACE, "workspace must be %zu-byte aligned", kAlign);
+    char *ws = static_cast<char *>(workspace);
+    SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
+                            sel_idx, sel_count, out, reinterpret_cast<float *>(ws + L.part_o_off),
+                            reinterpret_cast<float *>(ws + L.part_ml_off),
+                            reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params, const void *q,
+                            const void *k_cache, const void *v_cache, const float *k_scale,
+                            const float *v_scale, const int32_t *block_table, const int32_t *seq_lens,
+                            const float *kbar, float *out, int32_t *sel_idx, int32_t *sel_count,
+                            float *scores_out, void *workspace, size_t workspace_bytes,
+                            spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    SP_TRY(check_params(params));
+    SP_TRY(check_cache_args(dims, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens));
+    if (!kbar || !out || !sel_idx || !sel_count)
+        return fail(SPATTN_ERR_INVALID_ARG, "kbar, out, sel_idx, sel_count are required");
+    if (((uintptr_t)kbar | (uintptr_t)out) & 15)
+        return fail(SPATTN_ERR_INVALID_ARG, "kbar and out must be 16-byte aligned");
+    const int32_t need = required_max_sel(dims, params);
+    if (dims->max_sel < need)
+        return fail(SPATTN_ERR_INVALID_ARG, "max_sel %d < required %d", dims->max_sel, need);
+    const DecodeLayout L = decode_layout(dims, scores_out == nullptr);
+    if (!workspace || workspace_bytes < L.total)
+        return fail(SPATTN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", workspace_bytes, L.total);
+    if ((uintptr_t)workspace & (kAlign - 1))
+        return fail(SPATTN_ERR_WORKSPACE, "workspace must be %zu-byte aligned", kAlign);
+    char *ws = static_cast<char *>(workspace);
+    float *scores = scores_out ? scores_out : reinterpret_cast<float *>(ws + L.scores_off);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    SP_TRY(launch_scores(dims, params, q, kbar, block_table, seq_lens, scores, st));
+    SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count, st));
+    SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
+                            sel_idx, sel_count, out, reinterpret_cast<float *>(ws + L.part_o_off),
+                            reinterpret_cast<float *>(ws + L.part_ml_off), st));
+    return ok();
+}
+
+const char *spattn_last_error(void) { return g_err.c_str(); }
+
+spattn_status spattn_get_device_status(int32_t *host_out, spattn_stream_t stream) {
+    if (!host_out) return fail(SPATTN_ERR_INVALID_ARG, "host_out is NULL");
+    SP_TRY(cuda_ok(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "cudaStreamSynchronize"));
+    int32_t v = 0;
+    SP_TRY(cuda_ok(cudaMemcpyFromSymbol(&v, g_status, sizeof v), "read status word"));
+    const int32_t zero = 0;
+    SP_TRY(cuda_ok(cudaMemcpyToSymbol(g_status, &zero, sizeof zero), "clear status word"));
+    *host_out = v;
+    return ok();
+}
+
+const char *spattn_version(void) { return "spattn 0.1 sm_100a"; }
+
+}  // extern "C"

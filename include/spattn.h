@@ -1,0 +1,234 @@
+/*
+ * spattn.h -- C ABI of libspattn: block-sparse decode attention over a paged
+ * KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * For every query the library keeps the attention-sink block and the local
+ * window blocks, scores the middle 64-token blocks against mean-pooled
+ * (compressed) keys, keeps the best middle blocks by top-k or top-p, and runs
+ * exact softmax attention over the kept blocks only.
+ *
+ * Sources of the operation (page titles as printed):
+ *   "Claude Opus 长上下文 KV Cache 稀疏注意力", §稀疏注意力与 KV Cache 压缩的工程实现
+ *     (block-level management, attention sink, local window, Top-P
+ *     selection of middle blocks) and the configuration table of
+ *     §可落地的配置参数与监控要点 (64-token blocks, 1 sink block, 2 local
+ *     blocks, 10-20 % retention);
+ *   "CSA + HCA 混合注意力机制", §4.1 (compress m tokens into one entry; plain
+ *     averaging as the parameter-free compressor), §4.2 (score every
+ *     compressed entry, top-k, attend over the selected entries only), §4.3
+ *     (window + uncompressed tail join the attention), §4.4 (block-sparse
+ *     pattern: score, select, softmax(q K_sel^T / sqrt(d)) V_sel), §2.3 (the
+ *     decode step appends K, V then reads them back; the read is the
+ *     bottleneck);
+ *   "Claude Code压缩上下文窗口的底层原理与性能优化实践", 算法流程 (mean-pooling merge);
+ *   "Claude Code 1M 上下文" (aicoding.csdn.net), §2(3) (FP8 KV storage).
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers into memory the caller owns, unless
+ *     stated otherwise.  The library allocates nothing; scratch memory is the
+ *     caller's `workspace`.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and never synchronises, except
+ *     spattn_get_device_status.
+ *   - Arguments are validated on the host before anything is enqueued; a bad
+ *     argument returns SPATTN_ERR_INVALID_ARG (or _UNSUPPORTED) and enqueues
+ *     nothing.  spattn_last_error() then describes it.
+ *   - Bad DATA found on the device (a block-table entry outside
+ *     [0, num_pages), a selected block past the request's end, a selection
+ *     longer than max_sel, a bounded wait that gave up) never traps: the
+ *     kernel skips the offending access, sets a bit in the device status
+ *     word, and the result is unspecified.  Read and clear the word with
+ *     spattn_get_device_status.
+ *   - No C++ exception crosses this interface.
+ *
+ * Layouts (row-major, innermost last):
+ *   q          bf16  [B][Tq][Hq][d]        query tokens; token t of request b
+ *                                         sits at position seq_lens[b]-Tq+t
+ *   k_cache    bf16 or fp8-e4m3fn bytes [num_pages][Hkv][P][d]   (HND pages)
+ *   v_cache    same as k_cache
+ *   k_scale    f32   [num_pages][Hkv]      fp8 only: value = code * scale
+ *   v_scale    f32   [num_pages][Hkv]
+ *   block_table int32 [B][max_blocks_per_seq]  logical block j -> page id
+ *   seq_lens   int32 [B]                   tokens in the cache, including
+ *                                         the Tq query tokens
+ *   kbar       f32   [num_pages][Hkv][d]   mean-pooled key of each page
+ *   scores     f32   [B][Tq][Hkv][max_blocks_per_seq]
+ *   sel_idx    int32 [B][Hkv][max_sel]     kept logical block ids, ascending
+ *   sel_count  int32 [B][Hkv]
+ *   out        f32   [B][Tq][Hq][d]
+ * Query head i reads KV head i / (Hq / Hkv).  d must be 128 and P must be 64.
+ */
+#ifndef SPATTN_H
+#define SPATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *spattn_stream_t;
+
+typedef enum {
+    SPATTN_OK = 0,
+    SPATTN_ERR_INVALID_ARG = 1,   /* bad pointer, size or parameter */
+    SPATTN_ERR_UNSUPPORTED = 2,   /* valid but not built (d != 128, P != 64, ...) */
+    SPATTN_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+    SPATTN_ERR_WORKSPACE = 4,     /* workspace missing or too small */
+    SPATTN_ERR_TIMEOUT = 5,       /* reserved for host-side waits */
+    SPATTN_ERR_DEVICE = 6         /* the device status word is non-zero */
+} spattn_status;
+
+/* Bits of the device status word. */
+#define SPATTN_DEV_BAD_PAGE      0x1   /* block-table entry outside [0, num_pages) */
+#define SPATTN_DEV_BAD_BLOCK     0x2   /* selected block id outside [0, nb) */
+#define SPATTN_DEV_SEL_OVERFLOW  0x4   /* a selection did not fit in max_sel */
+#define SPATTN_DEV_WAIT_TIMEOUT  0x8   /* a bounded pipeline wait gave up */
+#define SPATTN_DEV_BAD_LEN       0x10  /* seq_len < 0 or > max_blocks_per_seq * P */
+
+typedef enum { SPATTN_KV_BF16 = 0, SPATTN_KV_FP8_E4M3 = 1 } spattn_kv_dtype;
+typedef enum { SPATTN_SEL_TOPK = 0, SPATTN_SEL_TOPP = 1 } spattn_sel_mode;
+
+typedef struct {
+    int32_t batch;              /* B >= 1 */
+    int32_t q_tokens;           /* Tq >= 1: query tokens per request (1 = decode) */
+    int32_t num_q_heads;        /* Hq, a multiple of Hkv; Tq * Hq / Hkv <= 64 */
+    int32_t num_kv_heads;       /* Hkv in [1, 16] */
+    int32_t head_dim;           /* d, must be 128 */
+    int32_t block_size;         /* P, must be 64 */
+    int32_t num_pages;          /* pages in the cache pool (>= 1) */
+    int32_t max_blocks_per_seq; /* columns of block_table and scores */
+    int32_t max_sel;            /* columns of sel_idx; >= spattn_required_max_sel() */
+    int32_t kv_dtype;           /* spattn_kv_dtype */
+} spattn_dims;
+
+typedef struct {
+    int32_t sink_blocks;        /* S >= 0: blocks [0, S) are always kept */
+    int32_t local_blocks;       /* W >= 0: the last W blocks are always kept */
+    int32_t mode;               /* spattn_sel_mode */
+    int32_t top_k;              /* top-k: k when > 0, else k = k_max */
+    float top_p;                /* top-p: mass threshold in (0, 1] */
+    float max_ratio;            /* cap k_max = floor(max_ratio * n_mid), in
+                                   [0, 1]; 0 means no cap (k_max = n_mid) */
+    float sm_scale;             /* softmax and score scale; 0 = 1/sqrt(d) */
+} spattn_params;
+
+/*
+ * Middle blocks of a request of nb = ceil(L / P) blocks are [S, nb - W);
+ * n_mid = max(0, nb - S - W).  Per query token the kept middle set is
+ *   top-k: the k = min(top_k > 0 ? top_k : k_max, k_max) best blocks, ranked
+ *          by score descending, equal scores by lower block id;
+ *   top-p: the shortest prefix of that ranking whose softmax probability
+ *          (softmax over the middle blocks' scores) reaches top_p, cut to
+ *          k_max blocks.
+ * The kept set of (b, h) is sink + local + the union over the Tq tokens.
+ */
+
+/* Columns sel_idx needs for these dims and parameters:
+ * min(max_blocks, S + W + min(n_mid, Tq * k)) at the longest request, with k
+ * the largest per-token middle count the parameters allow.  Returns -1 on
+ * invalid arguments. */
+int32_t spattn_required_max_sel(const spattn_dims *dims, const spattn_params *params);
+
+/*
+ * spattn_compress_keys -- mean-pooled key of each block.
+ * ("Claude Code压缩上下文窗口的底层原理与性能优化实践", 算法流程, 均值池化合并;
+ *  "CSA + HCA 混合注意力机制" §4.1.)
+ *
+ * kbar[page][h][:] = mean over the filled tokens of block j of K (dequantised
+ * with k_scale for fp8), for page = block_table[b][j], in fp32.  A block
+ * holds min(P, L - j*P) tokens.  With old_lens == NULL every block of every
+ * request is recomputed; otherwise only the blocks that hold a token of
+ * [old_lens[b], seq_lens[b]) (the tokens appended since the last call).
+ * k_scale may be NULL for bf16 caches.  Pages not touched keep their value.
+ */
+spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache,
+                                   const float *k_scale, const int32_t *block_table,
+                                   const int32_t *old_lens, const int32_t *seq_lens,
+                                   float *kbar, spattn_stream_t stream);
+
+/*
+ * spattn_block_scores -- score every middle block.
+ * ("CSA + HCA 混合注意力机制" §4.2 Lightning Indexer steps 3-4 and §4.4 step 1.)
+ *
+ * scores[b][t][h][j] = sm_scale * (qbar . kbar[block_table[b][j]][h]) for
+ * middle blocks j, where qbar is the fp32 mean of the Hq/Hkv query rows of
+ * token t that share KV head h; -inf in every other column (sink, local,
+ * past the end).  fp32 arithmetic throughout.
+ */
+spattn_status spattn_block_scores(const spattn_dims *dims, const spattn_params *params,
+                                  const void *q, const float *kbar,
+                                  const int32_t *block_table, const int32_t *seq_lens,
+                                  float *scores, spattn_stream_t stream);
+
+/*
+ * spattn_select -- sink + local + top-k / top-p middle blocks per (b, h).
+ * ("Claude Opus 长上下文 KV Cache 稀疏注意力", §稀疏注意力与 KV Cache 压缩的工程实现;
+ *  "CSA + HCA 混合注意力机制" §4.4 step 3.)
+ *
+ * Reads scores as written by spattn_block_scores (only the middle columns
+ * are read) and writes the ascending kept block ids of (b, h) to
+ * sel_idx[b][h][0 .. sel_count[b][h]).  Top-p probabilities and their running
+ * sum are fp32.
+ */
+spattn_status spattn_select(const spattn_dims *dims, const spattn_params *params,
+                            const float *scores, const int32_t *seq_lens,
+                            int32_t *sel_idx, int32_t *sel_count, spattn_stream_t stream);
+
+/* Bytes of workspace spattn_decode / spattn_decode_selected need (split-KV
+ * partial results and, for spattn_decode without scores_out, the scores).
+ * Returns 0 on invalid arguments. */
+size_t spattn_decode_workspace_size(const spattn_dims *dims, const spattn_params *params);
+
+/*
+ * spattn_decode_selected -- exact attention over a given selection.
+ * ("CSA + HCA 混合注意力机制" §2.1 and §4.4 step 4: softmax(q K_sel^T/sqrt(d)) V_sel.)
+ *
+ * out[b][t][i][:] = sum over tokens tau of the kept blocks of (b, h = i/G)
+ * with position tau < seq_lens[b] and tau <= seq_lens[b] - Tq + t of
+ * softmax_tau(sm_scale * q . k_tau) * v_tau, in fp32 (bf16 or fp8 inputs,
+ * fp32 accumulation; split-KV partials merged by their log-sum-exp).
+ * A row with no visible token is all zeros.  sel_idx / sel_count as written
+ * by spattn_select (any ascending or unordered list of distinct ids works).
+ */
+spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_params *params,
+                                     const void *q, const void *k_cache, const void *v_cache,
+                                     const float *k_scale, const float *v_scale,
+                                     const int32_t *block_table, const int32_t *seq_lens,
+                                     const int32_t *sel_idx, const int32_t *sel_count,
+                                     float *out, void *workspace, size_t workspace_bytes,
+                                     spattn_stream_t stream);
+
+/*
+ * spattn_decode -- the whole decode step after the cache append:
+ * block scores, selection, sparse attention and the split merge.
+ * kbar must be current (spattn_compress_keys after each append).
+ * sel_idx / sel_count receive the selection; scores_out (optional, may be
+ * NULL) receives the block scores, otherwise they live in the workspace.
+ */
+spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params,
+                            const void *q, const void *k_cache, const void *v_cache,
+                            const float *k_scale, const float *v_scale,
+                            const int32_t *block_table, const int32_t *seq_lens,
+                            const float *kbar, float *out, int32_t *sel_idx,
+                            int32_t *sel_count, float *scores_out, void *workspace,
+                            size_t workspace_bytes, spattn_stream_t stream);
+
+/* Message for the last failed call on this host thread ("" if none). */
+const char *spattn_last_error(void);
+
+/* Synchronises `stream`, copies the current device's status word to
+ * *host_out (host pointer) and clears it.  Returns SPATTN_OK when the copy
+ * worked (whatever the word holds). */
+spattn_status spattn_get_device_status(int32_t *host_out, spattn_stream_t stream);
+
+/* Library version string, e.g. "spattn 0.1 sm_100a". */
+const char *spattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPATTN_H */

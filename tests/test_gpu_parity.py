@@ -1,0 +1,156 @@
+"""CUDA library vs float64 oracle, element by element, on the same seeded bytes.
+
+Small cases run every request through the oracle; the five full-size
+workloads (the benchmark's launch configuration) are checked on sampled
+requests, each request through the oracle in full.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_kv_spattn_b200 import spattn
+from block_sparse_kv_spattn_b200.workloads import WORKLOADS, Workload, make_inputs
+from tests.cases import SMALL_CASES
+from tests.parity import compare, lib_params, run_library
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda):
+    spattn.load()
+    spattn.device_status()  # clear any stale bit
+
+
+@pytest.mark.parametrize("w", SMALL_CASES, ids=lambda w: w.name)
+def test_small_case_parity(w):
+    inp = make_inputs(w, device="cuda")
+    gpu = run_library(inp)
+    s = compare(inp, gpu)
+    assert s["exact_rows"] + s["replayed_rows"] == w.batch * w.num_kv_heads
+
+
+FULL = {
+    "tiny_4k_gqa4": [0],
+    "decode_128k_b8": [0, 7],
+    "ragged_b32": None,          # shortest and longest request, chosen below
+    "decode_1m_mqa": [1],
+    "chunk16_fp8_512k": [2],
+}
+
+
+@pytest.mark.parametrize("name", list(FULL), ids=list(FULL))
+def test_full_size_sampled_parity(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w, device="cuda")
+    gpu = run_library(inp)
+    reqs = FULL[name]
+    if reqs is None:
+        sl = inp["seq_lens"].cpu()
+        reqs = [int(sl.argmin()), int(sl.argmax())]
+    s = compare(inp, gpu, requests=reqs)
+    assert s["out_err"] <= (2e-2 if w.kv_fp8 else 2e-3)
+    # every request's counts obey the rule, sampled or not
+    cnt = gpu["sel_count"].cpu().numpy()
+    assert cnt.max() <= gpu["max_sel"]
+
+
+def test_needles_are_recalled_at_1m():
+    """All planted needle blocks sit far above the noise: every one is kept."""
+    w = WORKLOADS["decode_1m_mqa"]
+    inp = make_inputs(w, device="cuda")
+    gpu = run_library(inp)
+    for b in range(w.batch):
+        kept = set(gpu["sel_idx"][b, 0, :gpu["sel_count"][b, 0]].tolist())
+        assert set(inp["boosted"][b][0].tolist()) <= kept
+
+
+def test_edge_lengths():
+    """Empty request, single token, exact block multiples, no middle blocks."""
+    w = Workload("edges", batch=7, q_tokens=1, num_q_heads=8, num_kv_heads=2, seq_len=64 * 8,
+                 structure="zipf", mode="topk", top_k=2, seed=21)
+    inp = make_inputs(w, device="cuda")
+    inp["seq_lens"] = torch.tensor([0, 1, 63, 64, 65, 64 * 3, 64 * 3 + 1], dtype=torch.int32,
+                                   device="cuda")
+    gpu = run_library(inp)
+    compare(inp, gpu)
+    assert int(gpu["sel_count"][0, 0]) == 0
+    assert torch.all(gpu["out"][0] == 0)
+
+
+def test_edge_lengths_chunk():
+    """Chunk of 4 query tokens with the causal mask inside short contexts."""
+    w = Workload("edges_chunk", batch=4, q_tokens=4, num_q_heads=8, num_kv_heads=2, seq_len=64 * 6,
+                 structure="zipf", mode="topk", top_k=1, seed=22)
+    inp = make_inputs(w, device="cuda")
+    inp["seq_lens"] = torch.tensor([4, 64, 67, 64 * 6], dtype=torch.int32, device="cuda")
+    gpu = run_library(inp)
+    compare(inp, gpu)
+
+
+def test_select_all_equals_dense_on_gpu():
+    """k = every middle block: the GPU output is dense attention (oracle)."""
+    w = Workload("dense", batch=2, q_tokens=1, num_q_heads=16, num_kv_heads=4, seq_len=64 * 37 + 9,
+                 structure="zipf", mode="topk", max_ratio=1.0, seed=23)
+    inp = make_inputs(w, device="cuda")
+    gpu = run_library(inp)
+    compare(inp, gpu)
+    nb = (w.seq_len + 63) // 64
+    assert torch.all(gpu["sel_count"] == nb)
+
+
+def test_incremental_compress_matches_full():
+    """Appending tokens and compressing only the touched blocks gives the
+    same compressed keys as recompressing everything."""
+    w = WORKLOADS["tiny_4k_gqa4"].replace(seq_len=64 * 22)
+    inp = make_inputs(w, device="cuda")
+    kc, bt = inp["k_cache"], inp["block_table"]
+    old = torch.tensor([64 * 20 + 10], dtype=torch.int32, device="cuda")
+    new = old + 60                                      # crosses into a new block
+    page = int(bt[0, (int(old[0]) + 59) // 64])
+    g = torch.Generator(device="cuda").manual_seed(5)
+    kc[int(bt[0, int(old[0]) // 64]), :, int(old[0]) % 64:] = torch.randn(
+        (kc.shape[1], 64 - int(old[0]) % 64, 128), generator=g, device="cuda").to(kc.dtype)
+    kc[page, :, :(int(new[0]) % 64)] = torch.randn(
+        (kc.shape[1], int(new[0]) % 64, 128), generator=g, device="cuda").to(kc.dtype)
+    full = torch.zeros((kc.shape[0], kc.shape[1], 128), device="cuda")
+    inc = torch.zeros_like(full)
+    spattn.compress_keys(kc, inp["k_scale"], bt, old, inc)            # before the append
+    spattn.compress_keys(kc, inp["k_scale"], bt, new, inc, old_lens=old)
+    spattn.compress_keys(kc, inp["k_scale"], bt, new, full)
+    assert spattn.device_status() == 0
+    nb = (int(new[0]) + 63) // 64
+    used = bt[0, :nb].long()
+    torch.testing.assert_close(inc[used], full[used], rtol=0, atol=0)
+
+
+def test_bad_page_sets_status_without_fault():
+    """A block-table entry outside the pool is skipped and reported."""
+    w = WORKLOADS["tiny_4k_gqa4"]
+    inp = make_inputs(w, device="cuda")
+    inp["block_table"] = inp["block_table"].clone()
+    inp["block_table"][0, 20] = inp["num_pages"] + 7
+    gpu = run_library(inp)
+    assert gpu["status"] & spattn.DEV_BAD_PAGE
+
+
+def test_decode_selected_with_given_selection():
+    """spattn_decode_selected over a hand-given (unsorted) selection."""
+    from tests.parity import subproblem  # noqa: F401  (same helpers)
+    import oracle
+    from tests.oracle_io import bits16, cache_bytes, dims_of, params_of
+    w = WORKLOADS["tiny_4k_gqa4"]
+    inp = make_inputs(w, device="cuda")
+    sel = torch.tensor([[[63, 0, 17, 5, 62, 40]] * 2], dtype=torch.int32, device="cuda")
+    cnt = torch.full((1, 2), 6, dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 1, 8, 128), device="cuda")
+    params = lib_params(w)
+    dims = spattn.dims_for(inp["q"], inp["k_cache"], inp["block_table"], 6)
+    ws = spattn.alloc_workspace(dims, params, "cuda")
+    spattn.decode_selected(inp["q"], inp["k_cache"], inp["v_cache"], inp["k_scale"], inp["v_scale"],
+                           inp["block_table"], inp["seq_lens"], sel, cnt, out, ws, params)
+    assert spattn.device_status() == 0
+    ref = oracle.attend(dims_of(inp, 6), params_of(w), bits16(inp["q"]), cache_bytes(inp["k_cache"]),
+                        cache_bytes(inp["v_cache"]), None, None, inp["block_table"].cpu().numpy(),
+                        inp["seq_lens"].cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy())
+    assert np.abs(out.double().cpu().numpy() - ref).max() <= 2e-3

@@ -16,15 +16,7 @@ import oracle
 from block_sparse_kv_spattn_b200.workloads import WORKLOADS, Workload, make_inputs
 from tests.oracle_io import bits16, dequant, dims_of, host_arrays, params_of, run_oracle
 
-SMALL_TOPP = Workload("small_topp", batch=2, q_tokens=1, num_q_heads=8, num_kv_heads=2,
-                      seq_len=64 * 40 + 17, structure="zipf", mode="topp", top_p=0.9,
-                      max_ratio=0.15, seed=11)
-SMALL_FP8_CHUNK = Workload("small_fp8_chunk", batch=2, q_tokens=4, num_q_heads=8, num_kv_heads=2,
-                           seq_len=64 * 30 + 5, kv_fp8=True, structure="zipf", mode="topk",
-                           max_ratio=0.12, seed=12)
-SMALL_RAGGED = Workload("small_ragged", batch=3, q_tokens=1, num_q_heads=4, num_kv_heads=1,
-                        seq_len=0, ragged=(100, 5000), structure="planted", n_planted=3,
-                        mode="topk", top_k=5, seed=13)
+from tests.cases import SMALL_FP8_CHUNK, SMALL_RAGGED, SMALL_TOPP
 
 
 @pytest.fixture(scope="module")
