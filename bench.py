@@ -140,13 +140,30 @@ def step_bytes(inp, sel_count: torch.Tensor) -> dict:
     return dict(kv=kv, kbar=kbar, q=q, out=out, total=kv + kbar + q + out, kept_block_heads=kept)
 
 
+def reduce_over_ranks(t: torch.Tensor, world: int) -> list:
+    """[times..., bytes, bytes]: the first three (timed totals) take the max
+    over ranks, the last two (bytes moved) the sum.  Every rank calls it."""
+    if world > 1:
+        mx = t[:3].clone()
+        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
+        sm = t[3:].clone()
+        torch.distributed.all_reduce(sm, op=torch.distributed.ReduceOp.SUM)
+        t = torch.cat([mx, sm])
+    return t.tolist()
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent batch."""
+    return base + 1000 * rank
+
+
 def run_native(args, rank, world, local_rank):
     from block_sparse_kv_spattn_b200 import spattn
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = WORKLOADS[args.workload]
-    inp = make_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    inp = make_inputs(w, device=dev, seed=rank_seed(w.seed, rank))
     q, kc, vc, ks, vs = inp["q"], inp["k_cache"], inp["v_cache"], inp["k_scale"], inp["v_scale"]
     bt, sl = inp["block_table"], inp["seq_lens"]
     params = spattn.Params(sink_blocks=w.sink_blocks, local_blocks=w.local_blocks, mode=w.mode,
@@ -207,6 +224,9 @@ def run_native(args, rank, world, local_rank):
               if hasattr(props, "pci_bus_id") else str(local_rank))
     with Clocks(smi_id) as clk:
         t_wall = time.perf_counter()
+        # hold the stream for ~50 ms so the host queues steps ahead of the
+        # device: the events then time device work, not host submission
+        torch.cuda._sleep(int(0.05 * props.clock_rate * 1e3))
         for i in range(K):
             flush.zero_()
             ev[i][0].record()
@@ -245,13 +265,7 @@ def run_native(args, rank, world, local_rank):
 
     t = torch.tensor([total_ms, sum(attn_ms), e2e_ms, float(bts["total"]), float(bts["kv"] + bts["q"] + bts["out"])],
                      dtype=torch.float64, device=dev)
-    if world > 1:
-        mx = t[:3].clone()
-        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
-        sm = t[3:].clone()
-        torch.distributed.all_reduce(sm, op=torch.distributed.ReduceOp.SUM)
-        t = torch.cat([mx, sm])
-    total_ms, attn_total_ms, e2e_total_ms, all_bytes, _ = t.tolist()
+    total_ms, attn_total_ms, e2e_total_ms, all_bytes, _ = reduce_over_ranks(t, world)
     if rank != 0:
         return None
     ms_per_step = total_ms / K

@@ -95,7 +95,7 @@ typedef struct {
     int32_t batch;              /* B >= 1 */
     int32_t q_tokens;           /* Tq >= 1: query tokens per request (1 = decode) */
     int32_t num_q_heads;        /* Hq, a multiple of Hkv; Tq * Hq / Hkv <= 64 */
-    int32_t num_kv_heads;       /* Hkv in [1, 16] */
+    int32_t num_kv_heads;       /* Hkv: 1, 2, 4, 8 or 16 */
     int32_t head_dim;           /* d, must be 128 */
     int32_t block_size;         /* P, must be 64 */
     int32_t num_pages;          /* pages in the cache pool (>= 1) */
