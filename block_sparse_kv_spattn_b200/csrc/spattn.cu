@@ -364,6 +364,34 @@ spattn_status check_cache_args(const spattn_dims *d, const void *q, const void *
     return SPATTN_OK;
 }
 
+// ------------------------------------------------ fixed scratch (no allocation)
+
+// Scratch of spattn_decode_selected_noalloc: a module-scope device array, one
+// instance on every device that loads this library, held until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::map<int, void *> g_noalloc_ptr;
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a stand-in, so the address is asked for once per
+// device (with that device current) and cached.
+spattn_status noalloc_scratch(void **out) {
+    int dev;
+    SP_TRY(cuda_ok(cudaGetDevice(&dev), "cudaGetDevice"));
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_noalloc_ptr.find(dev);
+    if (it != g_noalloc_ptr.end()) {
+        *out = it->second;
+        return SPATTN_OK;
+    }
+    void *p = nullptr;
+    SP_TRY(cuda_ok(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)"));
+    g_noalloc_ptr[dev] = p;
+    *out = p;
+    return SPATTN_OK;
+}
+
 }  // namespace
 
 // ================================================================ C ABI
@@ -458,6 +486,34 @@ spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_param
     if ((uintptr_t)workspace & (kAlign - 1))
         return fail(SPATTN_ERR_WORKSPACE, "workspace must be %zu-byte aligned", kAlign);
     char *ws = static_cast<char *>(workspace);
+    SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
+                            sel_idx, sel_count, out, reinterpret_cast<float *>(ws + L.part_o_off),
+                            reinterpret_cast<float *>(ws + L.part_ml_off),
+                            reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+spattn_status spattn_decode_selected_noalloc(const spattn_dims *dims, const spattn_params *params,
+                                             const void *q, const void *k_cache, const void *v_cache,
+                                             const float *k_scale, const float *v_scale,
+                                             const int32_t *block_table, const int32_t *seq_lens,
+                                             const int32_t *sel_idx, const int32_t *sel_count, float *out,
+                                             spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    SP_TRY(check_params(params));
+    SP_TRY(check_cache_args(dims, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens));
+    if (!sel_idx || !sel_count || !out)
+        return fail(SPATTN_ERR_INVALID_ARG, "sel_idx, sel_count, out are required");
+    if ((uintptr_t)out & 15) return fail(SPATTN_ERR_INVALID_ARG, "out must be 16-byte aligned");
+    const DecodeLayout L = decode_layout(dims, false);
+    if (L.total > kNoAllocScratchBytes)
+        return fail(SPATTN_ERR_UNSUPPORTED,
+                    "these dims need %zu bytes of scratch; the built-in scratch holds %zu bytes "
+                    "(use spattn_decode_selected with a workspace)",
+                    L.total, kNoAllocScratchBytes);
+    void *scratch = nullptr;
+    SP_TRY(noalloc_scratch(&scratch));
+    char *ws = static_cast<char *>(scratch);
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
                             sel_idx, sel_count, out, reinterpret_cast<float *>(ws + L.part_o_off),
                             reinterpret_cast<float *>(ws + L.part_ml_off),

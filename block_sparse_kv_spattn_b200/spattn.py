@@ -33,7 +33,8 @@ SEL_TOPK, SEL_TOPP = 0, 1
 
 EXPORTS = ("spattn_required_max_sel", "spattn_compress_keys", "spattn_block_scores",
            "spattn_select", "spattn_decode_workspace_size", "spattn_decode_selected",
-           "spattn_decode", "spattn_last_error", "spattn_get_device_status", "spattn_version")
+           "spattn_decode", "spattn_last_error", "spattn_get_device_status", "spattn_version",
+           "spattn_decode_selected_noalloc")
 
 
 class SpattnError(RuntimeError):
@@ -95,6 +96,7 @@ def load() -> ctypes.CDLL:
         "spattn_last_error": ([], ctypes.c_char_p),
         "spattn_get_device_status": ([P, P], ctypes.c_int),
         "spattn_version": ([], ctypes.c_char_p),
+        "spattn_decode_selected_noalloc": ([P] * 13, ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -184,6 +186,18 @@ def decode_selected(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens
         _p(k_scale) if fp8 else None, _p(v_scale) if fp8 else None, _p(block_table),
         _p(seq_lens), _p(sel_idx), _p(sel_count), _p(out), _p(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def decode_selected_noalloc(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, sel_idx,
+                            sel_count, out, params: Params, stream=None):
+    """decode_selected with the library's built-in scratch instead of a
+    workspace: for callers that cannot allocate device memory at the call."""
+    dims = dims_for(q, k_cache, block_table, sel_idx.shape[-1])
+    fp8 = dims.kv_dtype == KV_FP8_E4M3
+    _check(load().spattn_decode_selected_noalloc(
+        ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(k_cache), _p(v_cache),
+        _p(k_scale) if fp8 else None, _p(v_scale) if fp8 else None, _p(block_table),
+        _p(seq_lens), _p(sel_idx), _p(sel_count), _p(out), _stream(stream)))
 
 
 def decode(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, kbar, out, sel_idx,

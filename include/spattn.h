@@ -202,6 +202,37 @@ spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_param
                                      spattn_stream_t stream);
 
 /*
+ * spattn_decode_selected_noalloc -- spattn_decode_selected without a
+ * caller-supplied workspace.  (Not a step of the method: the pages have no
+ * counterpart; it only changes where the scratch memory lives.)
+ *
+ * For callers that cannot allocate device memory at the point of the call:
+ * code running inside a host framework that owns every device allocation
+ * (an engine plugin, a caching allocator that must not be bypassed), code
+ * between the start and end of a CUDA stream capture, or latency-critical
+ * loops that must not pay for an allocation or for the implicit device
+ * synchronisation of freeing one.  The split-KV partial results go to a
+ * fixed scratch array built into the library (8 MiB, a module-scope device
+ * array present on every GPU that loads the library until the process
+ * exits).  Arguments, layouts and results are those of
+ * spattn_decode_selected; dims whose partial results need more than 8 MiB
+ * (slots x rows x (d + 2) x 4 bytes, slots = 320 + B * Hkv) are rejected with
+ * SPATTN_ERR_UNSUPPORTED before anything is enqueued.  No allocation call is
+ * made.  The first call on each device looks up the array's device address
+ * (a host-side CUDA runtime call), so make that first call before any stream
+ * capture.  Every call on a device shares the one array and leaves its
+ * contents behind; calls whose executions overlap on the GPU (different
+ * streams, or graphs replayed concurrently) race on it and give undefined
+ * results, so serialise them.
+ */
+spattn_status spattn_decode_selected_noalloc(const spattn_dims *dims, const spattn_params *params,
+                                             const void *q, const void *k_cache, const void *v_cache,
+                                             const float *k_scale, const float *v_scale,
+                                             const int32_t *block_table, const int32_t *seq_lens,
+                                             const int32_t *sel_idx, const int32_t *sel_count,
+                                             float *out, spattn_stream_t stream);
+
+/*
  * spattn_decode -- the whole decode step after the cache append:
  * block scores, selection, sparse attention and the split merge.
  * kbar must be current (spattn_compress_keys after each append).
