@@ -20,14 +20,24 @@ struct CompressArgs {
     int hkv, num_pages, max_blocks;
 };
 
-// Grid (gx, B); block = Hkv * 16 threads: thread (h, chunk) owns 8 columns
-// of KV head h.  CTA x walks the touched blocks of request y with stride gx.
-// Four interleaved fp32 partial sums per column keep the rounding error of
-// the 64-term sum near that of a depth-5 tree.
-template <bool FP8>
-__global__ void compress_keys_kernel(CompressArgs a) {
+// Token groups per CTA so that a CTA has up to 512 threads.
+__host__ __device__ constexpr int compress_groups(int hkv) {
+    return 512 / (hkv * 16) < 8 ? 512 / (hkv * 16) : 8;
+}
+
+// Grid (gx, B); block = TG * Hkv * 16 threads: thread (g, h, chunk) sums 8
+// columns of KV head h over the tokens t = g, g + TG, ... of a block (all its
+// loads issued together), and the TG partial sums are added in a fixed order
+// through shared memory.  CTA x walks the touched blocks of request y with
+// stride gx.
+template <bool FP8, int TG>
+__global__ void __launch_bounds__(512) compress_keys_kernel(CompressArgs a) {
+    constexpr int TPG = kBlock / TG;  // tokens per group
+    extern __shared__ float4 part4[];  // [TG][Hkv*16][2] float4
     const int b = blockIdx.y;
-    const int h = threadIdx.x >> 4, chunk = threadIdx.x & 15;
+    const int lanes = a.hkv * 16;
+    const int hc = threadIdx.x % lanes, g = threadIdx.x / lanes;
+    const int h = hc >> 4, chunk = hc & 15;
     const int L = a.seq_lens[b];
     if (L < 0 || L > a.max_blocks * kBlock) {
         if (threadIdx.x == 0 && blockIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
@@ -49,40 +59,43 @@ __global__ void compress_keys_kernel(CompressArgs a) {
         }
         const int filled = min(kBlock, L - j * kBlock);
         const int64_t tile = ((int64_t)page * a.hkv + h) * kBlock * kHeadDim;
-        float s[4][8];
+        float s[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int c = 0; c < 8; ++c) s[c] = 0.f;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) s[q][c] = 0.f;
-        for (int t0 = 0; t0 < filled; t0 += 4) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int t = t0 + q;
-                if (t < filled) {
-                    float f[8];
-                    if (FP8) {
-                        uint2 u = *reinterpret_cast<const uint2 *>(a.k_cache + tile + t * kHeadDim +
-                                                                   chunk * 8);
-                        e4m3x8_to_f32(u, f);
-                    } else {
-                        uint4 u = *reinterpret_cast<const uint4 *>(
-                            a.k_cache + 2 * (tile + t * kHeadDim + chunk * 8));
-                        bf16x8_to_f32(u, f);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) s[q][c] += f[c];
+        for (int k = 0; k < TPG; ++k) {
+            const int t = g + k * TG;
+            if (t < filled) {
+                float f[8];
+                if (FP8) {
+                    const uint2 u = *reinterpret_cast<const uint2 *>(a.k_cache + tile + t * kHeadDim + chunk * 8);
+                    e4m3x8_to_f32(u, f);
+                } else {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(a.k_cache + 2 * (tile + t * kHeadDim + chunk * 8));
+                    bf16x8_to_f32(u, f);
                 }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) s[c] += f[c];
             }
         }
-        const float sc = FP8 ? a.k_scale[(int64_t)page * a.hkv + h] : 1.f;
-        float r[8];
+        part4[(g * lanes + hc) * 2 + 0] = make_float4(s[0], s[1], s[2], s[3]);
+        part4[(g * lanes + hc) * 2 + 1] = make_float4(s[4], s[5], s[6], s[7]);
+        __syncthreads();
+        if (g == 0) {
+            float4 x = part4[hc * 2], y = part4[hc * 2 + 1];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-            r[c] = (((s[0][c] + s[1][c]) + (s[2][c] + s[3][c])) * sc) / (float)filled;
-        float4 *dst = reinterpret_cast<float4 *>(a.kbar + ((int64_t)page * a.hkv + h) * kHeadDim +
-                                                 chunk * 8);
-        dst[0] = make_float4(r[0], r[1], r[2], r[3]);
-        dst[1] = make_float4(r[4], r[5], r[6], r[7]);
+            for (int gg = 1; gg < TG; ++gg) {
+                const float4 u = part4[(gg * lanes + hc) * 2], v = part4[(gg * lanes + hc) * 2 + 1];
+                x.x += u.x; x.y += u.y; x.z += u.z; x.w += u.w;
+                y.x += v.x; y.y += v.y; y.z += v.z; y.w += v.w;
+            }
+            const float sc = FP8 ? a.k_scale[(int64_t)page * a.hkv + h] : 1.f;
+            const float n = (float)filled;
+            float4 *dst = reinterpret_cast<float4 *>(a.kbar + ((int64_t)page * a.hkv + h) * kHeadDim + chunk * 8);
+            dst[0] = make_float4(x.x * sc / n, x.y * sc / n, x.z * sc / n, x.w * sc / n);
+            dst[1] = make_float4(y.x * sc / n, y.y * sc / n, y.z * sc / n, y.w * sc / n);
+        }
+        __syncthreads();
     }
 }
 

@@ -18,16 +18,19 @@ struct ScoresArgs {
     const int32_t *block_table;
     const int32_t *seq_lens;
     float *scores;            // [B][Tq][Hkv][max_blocks]
-    int tq, hq, num_pages, max_blocks, sink, local;
+    int tq, hq, num_pages, max_blocks, sink, local, bpc;
     float scale;
 };
 
-constexpr int kScoreThreads = 256;
-constexpr int kScoreBlocksPerCta = 64;
+constexpr int kScoreThreads = 128;
+
+// Blocks per CTA: small CTAs (many resident per SM, many loads in flight)
+// unless the query rows make the per-CTA q-bar prologue heavy.
+__host__ __device__ constexpr int score_blocks_per_cta(int rows) { return rows <= 16 ? 16 : 64; }
 
 // Sum of v[0..7] over the 32 lanes, scattered: afterwards lane l holds the
-// full sum of element (l >> 2) & 7 in v[0].  Butterfly halving at offsets 16,
-// 8, 4 (each lane keeps the half named by its offset bit), then plain xor
+// full sum of element (l >> 2) & 7.  Butterfly halving at offsets 16, 8, 4
+// (each lane keeps the half named by its offset bit), then plain xor
 // reductions at 2 and 1: 9 shuffles for 8 warp sums.
 __device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
     const int lane = threadIdx.x & 31;
@@ -49,18 +52,22 @@ __device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
     return r;
 }
 
-// Grid (ceil(max_blocks / 64), B).  Dynamic shared memory:
-// qbar [Tq][HKV][D] fp32 followed by a [Tq*HKV][64] fp32 output tile.
+// Grid (ceil(max_blocks / bpc), B), kScoreThreads threads.  Dynamic shared
+// memory: qbar [Tq][HKV][D] fp32, then a [Tq*HKV][bpc] output tile.
+// Warp w takes blocks w, w + 4, ... of the CTA's range, BIF of them at a
+// time with all their compressed-key loads issued together.
 template <int HKV>
 __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs a) {
+    constexpr int BIF = HKV >= 16 ? 1 : (HKV >= 8 ? 2 : 4);
+    constexpr int NW = kScoreThreads / 32;
     extern __shared__ float4 smem_f4[];
     float *qbar = reinterpret_cast<float *>(smem_f4);
-    float *tile = qbar + a.tq * HKV * kHeadDim;
+    const int rows = a.tq * HKV;
+    float *tile = qbar + rows * kHeadDim;
     const int b = blockIdx.y;
-    const int j0 = blockIdx.x * kScoreBlocksPerCta;
+    const int j0 = blockIdx.x * a.bpc;
     const int G = a.hq / HKV;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int rows = a.tq * HKV;
 
     int L = a.seq_lens[b];
     if (L < 0 || L > a.max_blocks * kBlock) {
@@ -69,62 +76,80 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     }
     const int nb = (L + kBlock - 1) / kBlock;
 
-    // 1. group-mean query rows
-    for (int idx = threadIdx.x; idx < rows * kHeadDim; idx += kScoreThreads) {
-        const int c = idx % kHeadDim, th = idx / kHeadDim;
+    // 1. group-mean query rows, 8 columns per task
+    for (int task = threadIdx.x; task < rows * (kHeadDim / 8); task += kScoreThreads) {
+        const int c8 = task % (kHeadDim / 8), th = task / (kHeadDim / 8);
         const int hh = th % HKV, t = th / HKV;
-        const uint16_t *qr = a.q + (((int64_t)b * a.tq + t) * a.hq + hh * G) * kHeadDim + c;
-        float s = 0.f;
-        for (int g = 0; g < G; ++g) s += __uint_as_float((uint32_t)qr[g * kHeadDim] << 16);
-        qbar[idx] = s / (float)G;
+        const uint16_t *qr = a.q + (((int64_t)b * a.tq + t) * a.hq + hh * G) * kHeadDim + c8 * 8;
+        float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int g = 0; g < G; ++g) {
+            float f[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qr + g * kHeadDim), f);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) s[c] += f[c];
+        }
+        float4 *dst = reinterpret_cast<float4 *>(qbar + th * kHeadDim + c8 * 8);
+        dst[0] = make_float4(s[0] / G, s[1] / G, s[2] / G, s[3] / G);
+        dst[1] = make_float4(s[4] / G, s[5] / G, s[6] / G, s[7] / G);
     }
     __syncthreads();
 
-    // 2. one warp per block j; lane owns columns [4*lane, 4*lane+4)
+    // 2. lane owns columns [4*lane, 4*lane+4) of every KV head's kbar row
     constexpr int HPC = HKV < 8 ? HKV : 8;      // heads per 8-value chunk
     constexpr int TPC = 8 / HPC;                // tokens per chunk
-    for (int jj = warp; jj < kScoreBlocksPerCta; jj += kScoreThreads / 32) {
-        const int j = j0 + jj;
-        if (j >= a.max_blocks) break;
-        const bool middle = j >= a.sink && j < nb - a.local;
-        if (!middle) {
-            for (int r = lane; r < rows; r += 32) tile[r * kScoreBlocksPerCta + jj] = -INFINITY;
-            continue;
-        }
-        const int page = a.block_table[(int64_t)b * a.max_blocks + j];
-        if (page < 0 || page >= a.num_pages) {
-            if (lane == 0) flag(SPATTN_DEV_BAD_PAGE);
-            for (int r = lane; r < rows; r += 32) tile[r * kScoreBlocksPerCta + jj] = -INFINITY;
-            continue;
-        }
-        float4 kv[HKV];
-        const float4 *kp = reinterpret_cast<const float4 *>(a.kbar + (int64_t)page * HKV * kHeadDim);
+    for (int jb = warp; jb < a.bpc; jb += NW * BIF) {
+        float4 kv[BIF][HKV];
+        bool mid[BIF];
 #pragma unroll
-        for (int hh = 0; hh < HKV; ++hh) kv[hh] = kp[hh * (kHeadDim / 4) + lane];
-
-        for (int t0 = 0; t0 < a.tq; t0 += TPC) {
-#pragma unroll
-            for (int h0 = 0; h0 < HKV; h0 += HPC) {
-                float v[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int tt = t0 + i / HPC, hh = h0 + i % HPC;
-                    float s = 0.f;
-                    if (tt < a.tq) {
-                        const float4 qv =
-                            reinterpret_cast<const float4 *>(qbar + (tt * HKV + hh) * kHeadDim)[lane];
-                        s = qv.x * kv[hh].x;
-                        s = fmaf(qv.y, kv[hh].y, s);
-                        s = fmaf(qv.z, kv[hh].z, s);
-                        s = fmaf(qv.w, kv[hh].w, s);
-                    }
-                    v[i] = s;
+        for (int f = 0; f < BIF; ++f) {
+            const int jj = jb + f * NW, j = j0 + jj;
+            mid[f] = jj < a.bpc && j < a.max_blocks && j >= a.sink && j < nb - a.local;
+            int page = -1;
+            if (mid[f]) {
+                page = a.block_table[(int64_t)b * a.max_blocks + j];
+                if (page < 0 || page >= a.num_pages) {
+                    if (lane == 0) flag(SPATTN_DEV_BAD_PAGE);
+                    mid[f] = false;
                 }
-                const float r = reduce_scatter8(v);
-                if ((lane & 3) == 0) {
-                    const int i = lane >> 2;
-                    const int tt = t0 + i / HPC, hh = h0 + i % HPC;
-                    if (tt < a.tq) tile[(tt * HKV + hh) * kScoreBlocksPerCta + jj] = r * a.scale;
+            }
+            if (mid[f]) {
+                const float4 *kp = reinterpret_cast<const float4 *>(a.kbar + (int64_t)page * HKV * kHeadDim);
+#pragma unroll
+                for (int hh = 0; hh < HKV; ++hh) kv[f][hh] = kp[hh * (kHeadDim / 4) + lane];
+            }
+        }
+#pragma unroll
+        for (int f = 0; f < BIF; ++f) {
+            const int jj = jb + f * NW;
+            if (jj >= a.bpc) break;
+            if (!mid[f]) {
+                for (int r = lane; r < rows; r += 32) tile[r * a.bpc + jj] = -INFINITY;
+                continue;
+            }
+            for (int t0 = 0; t0 < a.tq; t0 += TPC) {
+#pragma unroll
+                for (int h0 = 0; h0 < HKV; h0 += HPC) {
+                    float v[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int tt = t0 + i / HPC, hh = h0 + i % HPC;
+                        float s = 0.f;
+                        if (tt < a.tq) {
+                            const float4 qv =
+                                reinterpret_cast<const float4 *>(qbar + (tt * HKV + hh) * kHeadDim)[lane];
+                            s = qv.x * kv[f][hh].x;
+                            s = fmaf(qv.y, kv[f][hh].y, s);
+                            s = fmaf(qv.z, kv[f][hh].z, s);
+                            s = fmaf(qv.w, kv[f][hh].w, s);
+                        }
+                        v[i] = s;
+                    }
+                    const float r = reduce_scatter8(v);
+                    if ((lane & 3) == 0) {
+                        const int i = lane >> 2;
+                        const int tt = t0 + i / HPC, hh = h0 + i % HPC;
+                        if (tt < a.tq) tile[(tt * HKV + hh) * a.bpc + jj] = r * a.scale;
+                    }
                 }
             }
         }
@@ -132,8 +157,8 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     __syncthreads();
 
     // 3. coalesced store of the tile
-    for (int idx = threadIdx.x; idx < rows * kScoreBlocksPerCta; idx += kScoreThreads) {
-        const int jj = idx % kScoreBlocksPerCta, r = idx / kScoreBlocksPerCta;
+    for (int idx = threadIdx.x; idx < rows * a.bpc; idx += kScoreThreads) {
+        const int jj = idx % a.bpc, r = idx / a.bpc;
         const int j = j0 + jj;
         if (j < a.max_blocks) {
             const int hh = r % HKV, t = r / HKV;

@@ -57,9 +57,17 @@ __device__ void radix_select(const SelectShared &sh, int n, int k, uint32_t &T, 
         const int nbins = pass < 2 ? 2048 : 1024;
         for (int i = threadIdx.x; i < 2048; i += blockDim.x) sh.hist[i] = 0;
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const uint32_t key = sh.keys[i];
-            if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & (nbins - 1)], 1u);
+        // scores crowd into few digits: lanes with equal digits add once
+        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+            const int i = i0 + threadIdx.x;
+            uint32_t digit = 0xffffffffu;
+            if (i < n) {
+                const uint32_t key = sh.keys[i];
+                if ((key & mask) == prefix) digit = (key >> shift) & (nbins - 1);
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, digit);
+            if (digit != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
+                atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
         }
         __syncthreads();
         // bins in descending digit order, two per thread
@@ -111,6 +119,28 @@ __device__ void for_each_chosen(const SelectShared &sh, int n, uint32_t T, int n
         const uint32_t key = sh.keys[i];
         if (key > T || (key == T && eq_before++ < need_eq)) fn(i, sel_before++);
     }
+}
+
+// Block-wide max of one uint32 per thread (every thread calls it).
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, int *tmp) {
+    v = __reduce_max_sync(0xffffffffu, v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = (int)v;
+    __syncthreads();
+    uint32_t r = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = max(r, (uint32_t)tmp[w]);
+    return r;
+}
+
+// Block-wide sum of one float per thread, added in a fixed order.
+__device__ __forceinline__ float block_sum_f(float v, float *tmp) {
+    v = warp_sum(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += tmp[w];
+    return r;
 }
 
 __device__ void bitonic_sort_desc(unsigned long long *buf, int N) {
@@ -187,11 +217,35 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
             __syncthreads();
             continue;
         }
-        // top-p
+        // top-p: probabilities are the softmax of the middle scores
         if (k_max <= 0) continue;
-        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) sh.keys[i] = float_key(row[i]);
-        __syncthreads();
+        uint32_t kmax_local = 0;
+        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) {
+            const uint32_t key = float_key(row[i]);
+            sh.keys[i] = key;
+            kmax_local = max(kmax_local, key);
+        }
+        const float smax = key_float(block_max_u32(kmax_local, sh.itmp));
+        float z = 0.f;
+        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) z += expf(key_float(sh.keys[i]) - smax);
+        const float Z = block_sum_f(z, sh.ftmp);
         const int kc = k_max;
+        uint32_t T = 0;
+        int need_eq = 0;
+        if (kc < n_mid) {
+            radix_select(sh, n_mid, kc, T, need_eq);
+            // mass of the k_max best blocks: below p, the cap decides alone
+            float mass = 0.f;
+            for_each_chosen(sh, n_mid, T, need_eq,
+                            [&](int i, int) { mass += expf(key_float(sh.keys[i]) - smax) / Z; });
+            mass = block_sum_f(mass, sh.ftmp);
+            if (mass < a.top_p) {
+                for_each_chosen(sh, n_mid, T, need_eq, [&](int i, int) { sh.flags[S + i] = 1; });
+                __syncthreads();
+                continue;
+            }
+        }
+        // the shortest prefix reaching p lies within the candidates: sort them
         int npow = 1;
         while (npow < kc) npow <<= 1;
         for (int i = threadIdx.x; i < npow; i += blockDim.x) sh.sortbuf[i] = 0ull;
@@ -200,32 +254,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
             const uint32_t j = (uint32_t)(S + i);
             sh.sortbuf[slot] = ((unsigned long long)sh.keys[i] << 32) | (0xffffffffu - j);
         };
-        if (kc < n_mid) {
-            uint32_t T;
-            int need_eq;
-            radix_select(sh, n_mid, kc, T, need_eq);
+        if (kc < n_mid)
             for_each_chosen(sh, n_mid, T, need_eq, put);
-        } else {
+        else
             for (int i = threadIdx.x; i < n_mid; i += blockDim.x) put(i, i);
-        }
         __syncthreads();
         bitonic_sort_desc(sh.sortbuf, npow);
-        const float smax = key_float((uint32_t)(sh.sortbuf[0] >> 32));
-        // Z = sum over every middle block of exp(s - smax)
-        float z = 0.f;
-        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) z += expf(key_float(sh.keys[i]) - smax);
-        z = warp_sum(z);
-        if ((threadIdx.x & 31) == 0) sh.ftmp[threadIdx.x >> 5] = z;
         if (threadIdx.x == 0) sh.misc[2] = kc;  // first crossing (default: all kc)
         __syncthreads();
-        if (threadIdx.x < 32) {
-            float zz = threadIdx.x < (blockDim.x >> 5) ? sh.ftmp[threadIdx.x] : 0.f;
-            zz = warp_sum(zz);
-            if (threadIdx.x == 0) sh.ftmp[39] = zz;
-        }
-        __syncthreads();
-        const float Z = sh.ftmp[39];
-        // running mass over the sorted candidates
         const int per = (kc + blockDim.x - 1) / blockDim.x;
         const int lo = min(kc, (int)threadIdx.x * per), hi = min(kc, lo + per);
         float local = 0.f;

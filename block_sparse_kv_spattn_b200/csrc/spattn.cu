@@ -180,11 +180,13 @@ struct DecodeLayout {
     size_t scores_off, scores_bytes, part_o_off, part_ml_off, total;
 };
 
+// Workspace: [scores] | partial outputs | partial (max, sum).  One partial
+// record of `rows` query rows per slot; (C_max + units) slots.
 DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
     DecodeLayout L{};
     const int64_t units = (int64_t)d->batch * d->num_kv_heads;
     const int64_t slots = kMaxAttnCtas + units;
-    const int rows = rows_of(d);
+    const int64_t rows = rows_of(d);
     size_t off = 0;
     L.scores_off = 0;
     L.scores_bytes = with_scores ? align_up((size_t)d->batch * d->q_tokens * d->num_kv_heads *
@@ -192,9 +194,9 @@ DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
                                  : 0;
     off += L.scores_bytes;
     L.part_o_off = off;
-    off += align_up((size_t)slots * rows * kHeadDim * sizeof(float));
+    off += align_up((size_t)(slots * rows) * kHeadDim * sizeof(float));
     L.part_ml_off = off;
-    off += align_up((size_t)slots * rows * 2 * sizeof(float));
+    off += align_up((size_t)(slots * rows) * 2 * sizeof(float));
     L.total = off;
     return L;
 }
@@ -218,10 +220,11 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     a.local = p->local_blocks;
     a.scale = sm_scale_of(p);
     const int rowsq = d->q_tokens * d->num_kv_heads;
-    const int smem = rowsq * (kHeadDim + kScoreBlocksPerCta) * (int)sizeof(float);
+    a.bpc = score_blocks_per_cta(rowsq);
+    const int smem = rowsq * (kHeadDim + a.bpc) * (int)sizeof(float);
     if (smem > kMaxSmem)
         return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_kv_heads = %d too large for block scores", rowsq);
-    dim3 grid((d->max_blocks_per_seq + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta, d->batch);
+    dim3 grid((d->max_blocks_per_seq + a.bpc - 1) / a.bpc, d->batch);
     const void *fn = nullptr;
     switch (d->num_kv_heads) {
         case 1: fn = (const void *)block_scores_kernel<1>; break;
@@ -275,22 +278,46 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
     return cuda_ok(cudaGetLastError(), "select launch");
 }
 
+std::map<std::pair<int, const void *>, int> g_occ;
+
+// Resident CTAs per SM of a kernel (queried once per device), capped at
+// `want`: the persistent grid is sized to what can actually be resident.
+spattn_status resident_ctas(const void *func, int threads, int smem, int want, int *out) {
+    int dev;
+    SP_TRY(cuda_ok(cudaGetDevice(&dev), "cudaGetDevice"));
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_occ.find({dev, func});
+    if (it == g_occ.end()) {
+        int n = 0;
+        SP_TRY(cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem),
+                       "cudaOccupancyMaxActiveBlocksPerMultiprocessor"));
+        it = g_occ.emplace(std::make_pair(dev, func), n).first;
+    }
+    *out = std::max(1, std::min(want, it->second));
+    return SPATTN_OK;
+}
+
 template <int RG, bool FP8>
-spattn_status launch_attn_t(const AttnArgs &a, int ctas, cudaStream_t st) {
+spattn_status launch_attn_t(AttnArgs &a, int sms, cudaStream_t st, int *ctas_out) {
     const int smem = attn_smem_bytes(FP8, RG);
-    SP_TRY(ensure_smem((const void *)attn_kernel<RG, FP8>, smem));
+    const void *fn = (const void *)attn_kernel<RG, FP8>;
+    SP_TRY(ensure_smem(fn, smem));
+    int per_sm;
+    SP_TRY(resident_ctas(fn, kAttnThreads, smem, attn_ctas_per_sm(RG), &per_sm));
+    const int ctas = std::min(kMaxAttnCtas, sms * per_sm);
     attn_kernel<RG, FP8><<<ctas, kAttnThreads, smem, st>>>(a);
+    *ctas_out = ctas;
     return cuda_ok(cudaGetLastError(), "attention launch");
 }
 
 template <bool FP8>
-spattn_status launch_attn_rg(int rg, const AttnArgs &a, int ctas, cudaStream_t st) {
+spattn_status launch_attn_rg(int rg, AttnArgs &a, int sms, cudaStream_t st, int *ctas) {
     switch (rg) {
-        case 1: return launch_attn_t<1, FP8>(a, ctas, st);
-        case 2: return launch_attn_t<2, FP8>(a, ctas, st);
-        case 4: return launch_attn_t<4, FP8>(a, ctas, st);
-        case 8: return launch_attn_t<8, FP8>(a, ctas, st);
-        case 16: return launch_attn_t<16, FP8>(a, ctas, st);
+        case 1: return launch_attn_t<1, FP8>(a, sms, st, ctas);
+        case 2: return launch_attn_t<2, FP8>(a, sms, st, ctas);
+        case 4: return launch_attn_t<4, FP8>(a, sms, st, ctas);
+        case 8: return launch_attn_t<8, FP8>(a, sms, st, ctas);
+        case 16: return launch_attn_t<16, FP8>(a, sms, st, ctas);
     }
     return fail(SPATTN_ERR_UNSUPPORTED, "row groups %d", rg);
 }
@@ -299,14 +326,12 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
                                const void *k_cache, const void *v_cache, const float *k_scale,
                                const float *v_scale, const int32_t *bt, const int32_t *sl,
                                const int32_t *sel_idx, const int32_t *sel_count, float *out,
-                               float *part_o, float *part_ml, cudaStream_t st) {
+                               char *ws, const DecodeLayout &L, cudaStream_t st) {
     const bool fp8 = d->kv_dtype == SPATTN_KV_FP8_E4M3;
     const int rows = rows_of(d);
     const int rg = rg_of(rows);
     int sms;
     SP_TRY(sm_count(&sms));
-    const int per_sm = rg > 8 ? 1 : 2;
-    const int ctas = std::min(kMaxAttnCtas, sms * per_sm);
     AttnArgs a;
     a.q = static_cast<const uint16_t *>(q);
     a.k_cache = static_cast<const uint8_t *>(k_cache);
@@ -317,8 +342,8 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     a.seq_lens = sl;
     a.sel_idx = sel_idx;
     a.sel_count = sel_count;
-    a.part_o = part_o;
-    a.part_ml = part_ml;
+    a.part_o = reinterpret_cast<float *>(ws + L.part_o_off);
+    a.part_ml = reinterpret_cast<float *>(ws + L.part_ml_off);
     a.tq = d->q_tokens;
     a.hq = d->num_q_heads;
     a.hkv = d->num_kv_heads;
@@ -329,11 +354,12 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     a.max_blocks = d->max_blocks_per_seq;
     a.max_sel = d->max_sel;
     a.qscale = sm_scale_of(p) * kLog2e;
-    SP_TRY(fp8 ? launch_attn_rg<true>(rg, a, ctas, st) : launch_attn_rg<false>(rg, a, ctas, st));
+    int ctas = 0;
+    SP_TRY(fp8 ? launch_attn_rg<true>(rg, a, sms, st, &ctas) : launch_attn_rg<false>(rg, a, sms, st, &ctas));
 
     MergeArgs m;
-    m.part_o = part_o;
-    m.part_ml = part_ml;
+    m.part_o = a.part_o;
+    m.part_ml = a.part_ml;
     m.sel_count = sel_count;
     m.out = out;
     m.batch = d->batch;
@@ -368,7 +394,7 @@ spattn_status check_cache_args(const spattn_dims *d, const void *q, const void *
 
 // Scratch of spattn_decode_selected_noalloc: a module-scope device array, one
 // instance on every device that loads this library, held until exit.
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::map<int, void *> g_noalloc_ptr;
@@ -391,6 +417,12 @@ spattn_status noalloc_scratch(void **out) {
     *out = p;
     return SPATTN_OK;
 }
+
+// The attention kernel's shared-memory regions are 16-byte aligned and the
+// two-CTA-per-SM shapes fit two CTAs (228 KiB per SM, 1 KiB reserved each).
+static_assert(attn_off_pbuf(false, 1) % 16 == 0 && attn_off_pbuf(true, 16) % 16 == 0, "layout");
+static_assert(2 * (attn_smem_bytes(false, 1) + 1024) <= 228 * 1024, "two CTAs per SM at one row group");
+static_assert(attn_smem_bytes(false, 16) <= 227 * 1024, "one CTA per SM at sixteen row groups");
 
 }  // namespace
 
@@ -425,12 +457,17 @@ spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache,
     a.max_blocks = dims->max_blocks_per_seq;
     const int gx = old_lens ? (dims->q_tokens + kBlock - 1) / kBlock + 1 : dims->max_blocks_per_seq;
     dim3 grid(gx, dims->batch);
-    const int threads = dims->num_kv_heads * 16;
+    const int tg = compress_groups(dims->num_kv_heads);
+    const int threads = tg * dims->num_kv_heads * 16;
+    const int smem = threads * 2 * (int)sizeof(float4);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (fp8)
-        compress_keys_kernel<true><<<grid, threads, 0, st>>>(a);
-    else
-        compress_keys_kernel<false><<<grid, threads, 0, st>>>(a);
+#define SP_COMPRESS(F, T) compress_keys_kernel<F, T><<<grid, threads, smem, st>>>(a)
+    if (fp8) {
+        if (tg == 8) SP_COMPRESS(true, 8); else if (tg == 4) SP_COMPRESS(true, 4); else SP_COMPRESS(true, 2);
+    } else {
+        if (tg == 8) SP_COMPRESS(false, 8); else if (tg == 4) SP_COMPRESS(false, 4); else SP_COMPRESS(false, 2);
+    }
+#undef SP_COMPRESS
     SP_TRY(cuda_ok(cudaGetLastError(), "compress_keys launch"));
     return ok();
 }
@@ -487,9 +524,7 @@ spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_param
         return fail(SPATTN_ERR_WORKSPACE, "workspace must be %zu-byte aligned", kAlign);
     char *ws = static_cast<char *>(workspace);
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
-                            sel_idx, sel_count, out, reinterpret_cast<float *>(ws + L.part_o_off),
-                            reinterpret_cast<float *>(ws + L.part_ml_off),
-                            reinterpret_cast<cudaStream_t>(stream)));
+                            sel_idx, sel_count, out, ws, L, reinterpret_cast<cudaStream_t>(stream)));
     return ok();
 }
 
@@ -515,9 +550,7 @@ spattn_status spattn_decode_selected_noalloc(const spattn_dims *dims, const spat
     SP_TRY(noalloc_scratch(&scratch));
     char *ws = static_cast<char *>(scratch);
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
-                            sel_idx, sel_count, out, reinterpret_cast<float *>(ws + L.part_o_off),
-                            reinterpret_cast<float *>(ws + L.part_ml_off),
-                            reinterpret_cast<cudaStream_t>(stream)));
+                            sel_idx, sel_count, out, ws, L, reinterpret_cast<cudaStream_t>(stream)));
     return ok();
 }
 
@@ -548,8 +581,7 @@ spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params
     SP_TRY(launch_scores(dims, params, q, kbar, block_table, seq_lens, scores, st));
     SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count, st));
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
-                            sel_idx, sel_count, out, reinterpret_cast<float *>(ws + L.part_o_off),
-                            reinterpret_cast<float *>(ws + L.part_ml_off), st));
+                            sel_idx, sel_count, out, ws, L, st));
     return ok();
 }
 

@@ -212,11 +212,11 @@ spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_param
  * between the start and end of a CUDA stream capture, or latency-critical
  * loops that must not pay for an allocation or for the implicit device
  * synchronisation of freeing one.  The split-KV partial results go to a
- * fixed scratch array built into the library (8 MiB, a module-scope device
+ * fixed scratch array built into the library (16 MiB, a module-scope device
  * array present on every GPU that loads the library until the process
  * exits).  Arguments, layouts and results are those of
- * spattn_decode_selected; dims whose partial results need more than 8 MiB
- * (slots x rows x (d + 2) x 4 bytes, slots = 320 + B * Hkv) are rejected with
+ * spattn_decode_selected; dims whose partial results need more than 16 MiB
+ * ((320 + B * Hkv) x (Tq * Hq / Hkv) x (d + 2) x 4 bytes) are rejected with
  * SPATTN_ERR_UNSUPPORTED before anything is enqueued.  No allocation call is
  * made.  The first call on each device looks up the array's device address
  * (a host-side CUDA runtime call), so make that first call before any stream
