@@ -4,7 +4,8 @@
                     [--workload NAME]
 
 One step is one pass of the whole decode path over the workload's batch:
-incremental key compression of each request's tail block, block scores,
+incremental key compression of each request's tail block (on a forked
+graph branch: the tail block is local, never scored), block scores,
 selection (sink + local + top-p/top-k), sparse attention and the split
 merge, all through the C ABI (captured once into CUDA graphs and replayed).
 Inputs are seeded synthetic data resident in HBM; L2 is flushed (a 512 MB
@@ -182,11 +183,20 @@ def run_native(args, rank, world, local_rank):
     ws = spattn.alloc_workspace(dims, params, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def front():   # append-side compression of the tail block, scores, selection
-        spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
-                             q_tokens=Tq)
+    # The step's appended tokens only touch the last local block(s): their
+    # compressed keys are never scored (local blocks are always kept), so the
+    # append-side compression runs on a forked branch beside scoring.
+    assert Tq <= (w.local_blocks - 1) * w.block_size + 1, "append would touch a middle block"
+    side = torch.cuda.Stream()
+
+    def front():   # scores + selection, with the tail block's compression beside them
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
+                                 q_tokens=Tq)
         spattn.block_scores(q, kbar, bt, sl, scores, params, k_cache=kc)
         spattn.select(scores, sl, sel_idx, sel_count, params, q=q, k_cache=kc, block_table=bt)
+        torch.cuda.current_stream().wait_stream(side)
 
     def attend():  # sparse attention + split merge
         spattn.decode_selected(q, kc, vc, ks, vs, bt, sl, sel_idx, sel_count, out, ws, params)

@@ -53,7 +53,9 @@ __device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
 }
 
 // Grid (ceil(max_blocks / bpc), B), kScoreThreads threads.  Dynamic shared
-// memory: qbar [Tq][HKV][D] fp32, then a [Tq*HKV][bpc] output tile.
+// memory: qbar [Tq][HKV][D] fp32, a [Tq*HKV][bpc] output tile, then the
+// page ids of the CTA's middle blocks (-1 elsewhere), read in the prologue
+// alongside the query rows.
 // Warp w takes blocks w, w + 4, ... of the CTA's range, BIF of them at a
 // time with all their compressed-key loads issued together.
 template <int HKV>
@@ -64,6 +66,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     float *qbar = reinterpret_cast<float *>(smem_f4);
     const int rows = a.tq * HKV;
     float *tile = qbar + rows * kHeadDim;
+    int *pages = reinterpret_cast<int *>(tile + rows * a.bpc);
     const int b = blockIdx.y;
     const int j0 = blockIdx.x * a.bpc;
     const int G = a.hq / HKV;
@@ -76,17 +79,38 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     }
     const int nb = (L + kBlock - 1) / kBlock;
 
-    // 1. group-mean query rows, 8 columns per task
+    // 1. page ids of the middle blocks, and group-mean query rows (8 columns per task)
+    for (int jj = threadIdx.x; jj < a.bpc; jj += kScoreThreads) {
+        const int j = j0 + jj;
+        int page = -1;
+        if (j < a.max_blocks && j >= a.sink && j < nb - a.local) {
+            page = a.block_table[(int64_t)b * a.max_blocks + j];
+            if (page < 0 || page >= a.num_pages) {
+                flag(SPATTN_DEV_BAD_PAGE);
+                page = -1;
+            }
+        }
+        pages[jj] = page;
+    }
     for (int task = threadIdx.x; task < rows * (kHeadDim / 8); task += kScoreThreads) {
         const int c8 = task % (kHeadDim / 8), th = task / (kHeadDim / 8);
         const int hh = th % HKV, t = th / HKV;
         const uint16_t *qr = a.q + (((int64_t)b * a.tq + t) * a.hq + hh * G) * kHeadDim + c8 * 8;
         float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int g = 0; g < G; ++g) {
-            float f[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qr + g * kHeadDim), f);
+        for (int g0 = 0; g0 < G; g0 += 4) {  // the group's rows are loaded 4 at a time
+            uint4 u[4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) s[c] += f[c];
+            for (int gg = 0; gg < 4; ++gg)
+                if (g0 + gg < G) u[gg] = *reinterpret_cast<const uint4 *>(qr + (g0 + gg) * kHeadDim);
+#pragma unroll
+            for (int gg = 0; gg < 4; ++gg) {
+                if (g0 + gg < G) {
+                    float f[8];
+                    bf16x8_to_f32(u[gg], f);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) s[c] += f[c];
+                }
+            }
         }
         float4 *dst = reinterpret_cast<float4 *>(qbar + th * kHeadDim + c8 * 8);
         dst[0] = make_float4(s[0] / G, s[1] / G, s[2] / G, s[3] / G);
@@ -102,16 +126,9 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
         bool mid[BIF];
 #pragma unroll
         for (int f = 0; f < BIF; ++f) {
-            const int jj = jb + f * NW, j = j0 + jj;
-            mid[f] = jj < a.bpc && j < a.max_blocks && j >= a.sink && j < nb - a.local;
-            int page = -1;
-            if (mid[f]) {
-                page = a.block_table[(int64_t)b * a.max_blocks + j];
-                if (page < 0 || page >= a.num_pages) {
-                    if (lane == 0) flag(SPATTN_DEV_BAD_PAGE);
-                    mid[f] = false;
-                }
-            }
+            const int jj = jb + f * NW;
+            const int page = jj < a.bpc ? pages[jj] : -1;
+            mid[f] = page >= 0;
             if (mid[f]) {
                 const float4 *kp = reinterpret_cast<const float4 *>(a.kbar + (int64_t)page * HKV * kHeadDim);
 #pragma unroll

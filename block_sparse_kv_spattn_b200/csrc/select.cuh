@@ -7,6 +7,13 @@
 // top-k of the scores.  Ranking: score descending, equal scores by lower
 // block id.  Top-p: the shortest prefix of the ranking whose softmax mass
 // (over the middle blocks) reaches p, cut to k_max = floor(ratio * n_mid).
+//
+// The top-k cut is found by bucketing the scores by value between the row's
+// min and max (2048 buckets, monotone in the score), so that every block in a
+// bucket above the crossing bucket is in, and ranking the few blocks of the
+// crossing bucket exactly by (score, index).  Rows whose crossing bucket is
+// crowded (many equal scores) fall back to a 3-pass radix select on the
+// order-preserving uint32 keys.
 #pragma once
 
 #include "common.cuh"
@@ -25,12 +32,17 @@ struct SelectArgs {
 };
 
 constexpr int kSelThreads = 1024;
+constexpr int kBuckets = 2048;
+constexpr int kCand = 256;     // largest crossing bucket ranked exactly
 
 struct SelectShared {
-    uint32_t *keys;            // [n_mid_cap]
     unsigned long long *sortbuf;  // [sort_cap]
-    uint32_t *hist;            // [2048]
-    int *itmp;                 // [40]
+    uint32_t *keys;            // [n_mid_cap]
+    uint32_t *hist;            // [kBuckets]
+    uint32_t *cand_key;        // [kCand]
+    int *cand_idx;             // [kCand]
+    int *cand_ok;              // [kCand]
+    int *itmp;                 // [72]
     float *ftmp;               // [40]
     int *misc;                 // [8]
     uint8_t *flags;            // [max_blocks]
@@ -40,24 +52,128 @@ __host__ __device__ inline size_t select_smem_bytes(int n_mid_cap, int sort_cap,
     size_t b = 0;
     b += (size_t)sort_cap * 8;
     b += (size_t)n_mid_cap * 4;
-    b += 2048 * 4 + 40 * 4 + 40 * 4 + 8 * 4;
+    b += kBuckets * 4 + 3 * kCand * 4 + 72 * 4 + 40 * 4 + 8 * 4;
     b += ((size_t)max_blocks + 15) / 16 * 16;
     return b;
 }
 
-// k-th largest key (1 <= k <= n) by a 3-pass most-significant-digit radix
-// select (11 + 11 + 10 bits).  Returns the key T and how many elements equal
-// to T belong to the top k (the rest of the top k is strictly greater).
-__device__ void radix_select(const SelectShared &sh, int n, int k, uint32_t &T, int &need_eq) {
+// ------------------------------------------------------------ block helpers
+
+// Block-wide max and min of one uint32 per thread (every thread calls it).
+__device__ __forceinline__ void block_minmax_u32(uint32_t vmax, uint32_t vmin, int *tmp, uint32_t &omax,
+                                                 uint32_t &omin) {
+    vmax = __reduce_max_sync(0xffffffffu, vmax);
+    vmin = __reduce_min_sync(0xffffffffu, vmin);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) {
+        tmp[threadIdx.x >> 5] = (int)vmax;
+        tmp[32 + (threadIdx.x >> 5)] = (int)vmin;
+    }
+    __syncthreads();
+    omax = 0;
+    omin = 0xffffffffu;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        omax = max(omax, (uint32_t)tmp[w]);
+        omin = min(omin, (uint32_t)tmp[32 + w]);
+    }
+}
+
+// Block-wide sum of one float per thread, added in a fixed order.
+__device__ __forceinline__ float block_sum_f(float v, float *tmp) {
+    v = warp_sum(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += tmp[w];
+    return r;
+}
+
+// Middle scores of a row -> order-preserving keys in shared memory.  The
+// row buffer has n_cap >= n readable columns, so the loads of a thread (8 at
+// a time) need not wait for n.  Returns the thread's max/min key over i < n.
+__device__ __forceinline__ void load_keys(const SelectShared &sh, const float *row, int n_cap,
+                                          const int *n_ptr, uint32_t &kmax, uint32_t &kmin) {
+    kmax = 0;
+    kmin = 0xffffffffu;
+    for (int i0 = threadIdx.x; i0 < n_cap; i0 += 8 * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * blockDim.x;
+            v[u] = i < n_cap ? row[i] : 0.f;
+        }
+        const int n = *n_ptr;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * blockDim.x;
+            if (i < n) {
+                const uint32_t key = float_key(v[u]);
+                sh.keys[i] = key;
+                kmax = max(kmax, key);
+                kmin = min(kmin, key);
+            }
+        }
+    }
+}
+
+// Histogram bins in descending order, 2048 / blockDim consecutive per
+// thread: the bin holding the kk-th element from the top, the count of all
+// elements in higher bins, and the bin's own count (misc[0..2]).
+__device__ void find_crossing(const SelectShared &sh, int nbins, int kk) {
+    const int bpt = kBuckets / blockDim.x;
+    const int p0 = threadIdx.x * bpt;
+    int mine = 0;
+    for (int q = 0; q < bpt; ++q)
+        if (p0 + q < nbins) mine += (int)sh.hist[nbins - 1 - p0 - q];
+    int tot;
+    int ex = block_excl_scan(mine, sh.itmp, &tot);
+    if (ex < kk && kk <= ex + mine) {
+        for (int q = 0; q < bpt; ++q) {
+            const int c = (int)sh.hist[nbins - 1 - p0 - q];
+            if (kk <= ex + c) {
+                sh.misc[0] = nbins - 1 - p0 - q;
+                sh.misc[1] = ex;
+                sh.misc[2] = c;
+                break;
+            }
+            ex += c;
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------- the cut
+
+// The top k of a row (1 <= k < n): either "bucket" form -- every element in
+// a bucket above `bstar`, plus the crossing bucket's candidates flagged in
+// cand_ok -- or "radix" form -- every key above T plus the first need_eq keys
+// equal to T by index.
+struct Cut {
+    bool bucket;
+    float smin, inv;
+    int bstar, ncand;
+    uint32_t T;
+    int need_eq, cnt_eq;
+};
+
+__device__ __forceinline__ int bucket_of(float s, float smin, float inv) {
+    const int b = (int)((s - smin) * inv);  // monotone non-decreasing in s
+    return min(max(b, 0), kBuckets - 1);
+}
+
+// k-th largest key by a 3-pass most-significant-digit radix select
+// (11 + 11 + 10 bits): the key T, how many keys equal to T belong to the
+// top k, and how many keys equal T in all.
+__device__ void radix_select(const SelectShared &sh, int n, int k, uint32_t &T, int &need_eq, int &cnt_eq) {
     uint32_t prefix = 0, mask = 0;
     int kk = k;
 #pragma unroll 1
     for (int pass = 0; pass < 3; ++pass) {
         const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
         const int nbins = pass < 2 ? 2048 : 1024;
-        for (int i = threadIdx.x; i < 2048; i += blockDim.x) sh.hist[i] = 0;
+        for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) sh.hist[i] = 0;
         __syncthreads();
-        // scores crowd into few digits: lanes with equal digits add once
         for (int i0 = 0; i0 < n; i0 += blockDim.x) {
             const int i = i0 + threadIdx.x;
             uint32_t digit = 0xffffffffu;
@@ -70,77 +186,94 @@ __device__ void radix_select(const SelectShared &sh, int n, int k, uint32_t &T, 
                 atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
         }
         __syncthreads();
-        // bins in descending digit order, two per thread
-        const int i0 = 2 * threadIdx.x;
-        const int c0 = i0 < nbins ? (int)sh.hist[nbins - 1 - i0] : 0;
-        const int c1 = i0 + 1 < nbins ? (int)sh.hist[nbins - 2 - i0] : 0;
-        int tot;
-        const int ex = block_excl_scan(c0 + c1, sh.itmp, &tot);
-        if (ex < kk && kk <= ex + c0) {
-            sh.misc[0] = nbins - 1 - i0;
-            sh.misc[1] = ex;
-        } else if (ex + c0 < kk && kk <= ex + c0 + c1) {
-            sh.misc[0] = nbins - 2 - i0;
-            sh.misc[1] = ex + c0;
-        }
-        __syncthreads();
+        find_crossing(sh, nbins, kk);
         prefix |= (uint32_t)sh.misc[0] << shift;
         mask |= (uint32_t)(nbins - 1) << shift;
         kk -= sh.misc[1];
+        cnt_eq = sh.misc[2];
         __syncthreads();
     }
     T = prefix;
     need_eq = kk;
 }
 
-// Visit the top-k set {key > T} + {the first need_eq keys == T by index} in
-// index order.  Each thread owns a contiguous index range; fn(i, slot) gets
-// the element's rank among the chosen elements in index order.
-template <typename Fn>
-__device__ void for_each_chosen(const SelectShared &sh, int n, uint32_t T, int need_eq, Fn fn) {
-    const int per = (n + blockDim.x - 1) / blockDim.x;
-    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
-    int ceq = 0, csel = 0;
-    for (int i = lo; i < hi; ++i) {
-        const uint32_t key = sh.keys[i];
-        ceq += key == T;
-    }
-    int tot;
-    int eq_before = block_excl_scan(ceq, sh.itmp, &tot);
-    {
-        int e = eq_before;
-        for (int i = lo; i < hi; ++i) {
-            const uint32_t key = sh.keys[i];
-            if (key > T || (key == T && e++ < need_eq)) ++csel;
+__device__ Cut find_cut(const SelectShared &sh, int n, int k, uint32_t kmax, uint32_t kmin) {
+    Cut cut{};
+    const float smax = key_float(kmax), smin = key_float(kmin);
+    if (isfinite(smax) && isfinite(smin) && smax > smin) {
+        cut.smin = smin;
+        cut.inv = (float)kBuckets / (smax - smin);
+        for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) sh.hist[i] = 0;
+        if (threadIdx.x == 0) sh.misc[3] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += blockDim.x)
+            atomicAdd(&sh.hist[bucket_of(key_float(sh.keys[i]), cut.smin, cut.inv)], 1u);
+        __syncthreads();
+        find_crossing(sh, kBuckets, k);
+        cut.bstar = sh.misc[0];
+        const int need = k - sh.misc[1], c = sh.misc[2];
+        if (c <= kCand) {
+            cut.bucket = true;
+            cut.ncand = c;
+            // gather the crossing bucket, then rank it exactly by (key desc, index asc)
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                const uint32_t key = sh.keys[i];
+                if (bucket_of(key_float(key), cut.smin, cut.inv) == cut.bstar) {
+                    const int slot = atomicAdd(&sh.misc[3], 1);
+                    sh.cand_key[slot] = key;
+                    sh.cand_idx[slot] = i;
+                }
+            }
+            __syncthreads();
+            for (int t = threadIdx.x; t < c; t += blockDim.x) {
+                const uint32_t kt = sh.cand_key[t];
+                const int it = sh.cand_idx[t];
+                int rank = 0;
+                for (int u = 0; u < c; ++u) {
+                    const uint32_t ku = sh.cand_key[u];
+                    rank += ku > kt || (ku == kt && sh.cand_idx[u] < it);
+                }
+                sh.cand_ok[t] = rank < need;
+            }
+            __syncthreads();
+            return cut;
         }
     }
-    int sel_before = block_excl_scan(csel, sh.itmp, &tot);
+    cut.bucket = false;
+    radix_select(sh, n, k, cut.T, cut.need_eq, cut.cnt_eq);
+    return cut;
+}
+
+// Visit the radix-form set {key > T} + {the first need_eq keys == T by
+// index} (contiguous index range per thread, one block scan).
+template <typename Fn>
+__device__ void for_each_radix_chosen(const SelectShared &sh, int n, uint32_t T, int need_eq, Fn fn) {
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+    int ceq = 0;
+    for (int i = lo; i < hi; ++i) ceq += sh.keys[i] == T;
+    int tot;
+    int eq_before = block_excl_scan(ceq, sh.itmp, &tot);
     for (int i = lo; i < hi; ++i) {
         const uint32_t key = sh.keys[i];
-        if (key > T || (key == T && eq_before++ < need_eq)) fn(i, sel_before++);
+        if (key > T || (key == T && eq_before++ < need_eq)) fn(i);
     }
 }
 
-// Block-wide max of one uint32 per thread (every thread calls it).
-__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, int *tmp) {
-    v = __reduce_max_sync(0xffffffffu, v);
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = (int)v;
-    __syncthreads();
-    uint32_t r = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = max(r, (uint32_t)tmp[w]);
-    return r;
-}
-
-// Block-wide sum of one float per thread, added in a fixed order.
-__device__ __forceinline__ float block_sum_f(float v, float *tmp) {
-    v = warp_sum(v);
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float r = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += tmp[w];
-    return r;
+// Every element of the cut, in no particular order, once: fn(i).
+template <typename Fn>
+__device__ void for_each_in_cut(const SelectShared &sh, int n, const Cut &cut, Fn fn) {
+    if (cut.bucket) {
+        for (int i = threadIdx.x; i < n; i += blockDim.x)
+            if (bucket_of(key_float(sh.keys[i]), cut.smin, cut.inv) > cut.bstar) fn(i);
+        for (int t = threadIdx.x; t < cut.ncand; t += blockDim.x)
+            if (sh.cand_ok[t]) fn(sh.cand_idx[t]);
+    } else if (cut.need_eq == cut.cnt_eq) {
+        for (int i = threadIdx.x; i < n; i += blockDim.x)
+            if (sh.keys[i] >= cut.T) fn(i);
+    } else {
+        for_each_radix_chosen(sh, n, cut.T, cut.need_eq, fn);
+    }
 }
 
 __device__ void bitonic_sort_desc(unsigned long long *buf, int N) {
@@ -161,7 +294,7 @@ __device__ void bitonic_sort_desc(unsigned long long *buf, int N) {
     }
 }
 
-// Grid (B * Hkv), block kSelThreads.
+// Grid (B * Hkv), block 256 / 512 / 1024 threads (longer rows, more).
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     extern __shared__ unsigned long long smem_u64[];
     SelectShared sh;
@@ -172,9 +305,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         sh.keys = reinterpret_cast<uint32_t *>(p);
         p += (size_t)a.n_mid_cap * 4;
         sh.hist = reinterpret_cast<uint32_t *>(p);
-        p += 2048 * 4;
+        p += kBuckets * 4;
+        sh.cand_key = reinterpret_cast<uint32_t *>(p);
+        p += kCand * 4;
+        sh.cand_idx = reinterpret_cast<int *>(p);
+        p += kCand * 4;
+        sh.cand_ok = reinterpret_cast<int *>(p);
+        p += kCand * 4;
         sh.itmp = reinterpret_cast<int *>(p);
-        p += 40 * 4;
+        p += 72 * 4;
         sh.ftmp = reinterpret_cast<float *>(p);
         p += 40 * 4;
         sh.misc = reinterpret_cast<int *>(p);
@@ -201,81 +340,72 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
 
     for (int t = 0; t < a.tq && n_mid > 0; ++t) {
         const float *row = a.scores + (((int64_t)b * a.tq + t) * a.hkv + h) * a.max_blocks + S;
-        if (a.mode == SPATTN_SEL_TOPK) {
-            if (k_topk >= n_mid) {
-                for (int i = threadIdx.x; i < n_mid; i += blockDim.x) sh.flags[S + i] = 1;
-                __syncthreads();
-                continue;
-            }
-            if (k_topk <= 0) continue;
-            for (int i = threadIdx.x; i < n_mid; i += blockDim.x) sh.keys[i] = float_key(row[i]);
+        const int k = a.mode == SPATTN_SEL_TOPK ? k_topk : k_max;
+        if (k <= 0) continue;
+        if (a.mode == SPATTN_SEL_TOPK && k >= n_mid) {
+            for (int i = threadIdx.x; i < n_mid; i += blockDim.x) sh.flags[S + i] = 1;
             __syncthreads();
-            uint32_t T;
-            int need_eq;
-            radix_select(sh, n_mid, k_topk, T, need_eq);
-            for_each_chosen(sh, n_mid, T, need_eq, [&](int i, int) { sh.flags[S + i] = 1; });
+            continue;
+        }
+        uint32_t kmax_l, kmin_l, kmax, kmin;
+        load_keys(sh, row, a.n_mid_cap, &n_mid, kmax_l, kmin_l);
+        block_minmax_u32(kmax_l, kmin_l, sh.itmp, kmax, kmin);
+        if (a.mode == SPATTN_SEL_TOPK) {
+            const Cut cut = find_cut(sh, n_mid, k, kmax, kmin);
+            for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });
             __syncthreads();
             continue;
         }
         // top-p: probabilities are the softmax of the middle scores
-        if (k_max <= 0) continue;
-        uint32_t kmax_local = 0;
-        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) {
-            const uint32_t key = float_key(row[i]);
-            sh.keys[i] = key;
-            kmax_local = max(kmax_local, key);
-        }
-        const float smax = key_float(block_max_u32(kmax_local, sh.itmp));
+        const float smax = key_float(kmax);
         float z = 0.f;
         for (int i = threadIdx.x; i < n_mid; i += blockDim.x) z += expf(key_float(sh.keys[i]) - smax);
         const float Z = block_sum_f(z, sh.ftmp);
-        const int kc = k_max;
-        uint32_t T = 0;
-        int need_eq = 0;
-        if (kc < n_mid) {
-            radix_select(sh, n_mid, kc, T, need_eq);
+        Cut cut{};
+        if (k < n_mid) {
+            cut = find_cut(sh, n_mid, k, kmax, kmin);
             // mass of the k_max best blocks: below p, the cap decides alone
-            float mass = 0.f;
-            for_each_chosen(sh, n_mid, T, need_eq,
-                            [&](int i, int) { mass += expf(key_float(sh.keys[i]) - smax) / Z; });
-            mass = block_sum_f(mass, sh.ftmp);
+            float m = 0.f;
+            for_each_in_cut(sh, n_mid, cut, [&](int i) { m += expf(key_float(sh.keys[i]) - smax); });
+            const float mass = block_sum_f(m, sh.ftmp) / Z;
             if (mass < a.top_p) {
-                for_each_chosen(sh, n_mid, T, need_eq, [&](int i, int) { sh.flags[S + i] = 1; });
+                for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });
                 __syncthreads();
                 continue;
             }
         }
-        // the shortest prefix reaching p lies within the candidates: sort them
+        // the shortest prefix reaching p lies within the k candidates: sort them
         int npow = 1;
-        while (npow < kc) npow <<= 1;
+        while (npow < k) npow <<= 1;
         for (int i = threadIdx.x; i < npow; i += blockDim.x) sh.sortbuf[i] = 0ull;
+        if (threadIdx.x == 0) sh.misc[4] = 0;
         __syncthreads();
-        auto put = [&](int i, int slot) {
-            const uint32_t j = (uint32_t)(S + i);
-            sh.sortbuf[slot] = ((unsigned long long)sh.keys[i] << 32) | (0xffffffffu - j);
+        auto put = [&](int i) {
+            const int slot = atomicAdd(&sh.misc[4], 1);
+            sh.sortbuf[slot] = ((unsigned long long)sh.keys[i] << 32) | (0xffffffffu - (uint32_t)(S + i));
         };
-        if (kc < n_mid)
-            for_each_chosen(sh, n_mid, T, need_eq, put);
+        if (k < n_mid)
+            for_each_in_cut(sh, n_mid, cut, put);
         else
-            for (int i = threadIdx.x; i < n_mid; i += blockDim.x) put(i, i);
+            for (int i = threadIdx.x; i < n_mid; i += blockDim.x) put(i);
         __syncthreads();
         bitonic_sort_desc(sh.sortbuf, npow);
-        if (threadIdx.x == 0) sh.misc[2] = kc;  // first crossing (default: all kc)
+        if (threadIdx.x == 0) sh.misc[5] = k;  // first crossing (default: all k)
         __syncthreads();
-        const int per = (kc + blockDim.x - 1) / blockDim.x;
-        const int lo = min(kc, (int)threadIdx.x * per), hi = min(kc, lo + per);
+        const int per = (k + blockDim.x - 1) / blockDim.x;
+        const int lo = min(k, (int)threadIdx.x * per), hi = min(k, lo + per);
         float local = 0.f;
         for (int i = lo; i < hi; ++i) local += expf(key_float((uint32_t)(sh.sortbuf[i] >> 32)) - smax) / Z;
         float c = block_incl_scan_f(local, sh.ftmp) - local;
         for (int i = lo; i < hi; ++i) {
             c += expf(key_float((uint32_t)(sh.sortbuf[i] >> 32)) - smax) / Z;
             if (c >= a.top_p) {
-                atomicMin(&sh.misc[2], i + 1);
+                atomicMin(&sh.misc[5], i + 1);
                 break;
             }
         }
         __syncthreads();
-        const int m = sh.misc[2];
+        const int m = sh.misc[5];
         for (int i = threadIdx.x; i < m; i += blockDim.x)
             sh.flags[0xffffffffu - (uint32_t)(sh.sortbuf[i] & 0xffffffffull)] = 1;
         __syncthreads();

@@ -203,6 +203,22 @@ DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
 
 // ------------------------------------------------------------- launches
 
+// Plain stream-ordered launch through cudaLaunchKernelEx.  (Programmatic
+// dependent launch was measured on this path and lost: an early-scheduled
+// successor takes SM resources the predecessor's tail still uses.)
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const void *q,
                             const float *kbar, const int32_t *bt, const int32_t *sl, float *scores,
                             cudaStream_t st) {
@@ -221,7 +237,7 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     a.scale = sm_scale_of(p);
     const int rowsq = d->q_tokens * d->num_kv_heads;
     a.bpc = score_blocks_per_cta(rowsq);
-    const int smem = rowsq * (kHeadDim + a.bpc) * (int)sizeof(float);
+    const int smem = rowsq * (kHeadDim + a.bpc) * (int)sizeof(float) + a.bpc * (int)sizeof(int);
     if (smem > kMaxSmem)
         return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_kv_heads = %d too large for block scores", rowsq);
     dim3 grid((d->max_blocks_per_seq + a.bpc - 1) / a.bpc, d->batch);
@@ -234,14 +250,15 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
         case 16: fn = (const void *)block_scores_kernel<16>; break;
     }
     SP_TRY(ensure_smem(fn, smem));
+    cudaError_t e = cudaSuccess;
     switch (d->num_kv_heads) {
-        case 1: block_scores_kernel<1><<<grid, kScoreThreads, smem, st>>>(a); break;
-        case 2: block_scores_kernel<2><<<grid, kScoreThreads, smem, st>>>(a); break;
-        case 4: block_scores_kernel<4><<<grid, kScoreThreads, smem, st>>>(a); break;
-        case 8: block_scores_kernel<8><<<grid, kScoreThreads, smem, st>>>(a); break;
-        case 16: block_scores_kernel<16><<<grid, kScoreThreads, smem, st>>>(a); break;
+        case 1: e = launch(block_scores_kernel<1>, grid, kScoreThreads, smem, st, a); break;
+        case 2: e = launch(block_scores_kernel<2>, grid, kScoreThreads, smem, st, a); break;
+        case 4: e = launch(block_scores_kernel<4>, grid, kScoreThreads, smem, st, a); break;
+        case 8: e = launch(block_scores_kernel<8>, grid, kScoreThreads, smem, st, a); break;
+        case 16: e = launch(block_scores_kernel<16>, grid, kScoreThreads, smem, st, a); break;
     }
-    return cuda_ok(cudaGetLastError(), "block_scores launch");
+    return cuda_ok(e, "block_scores launch");
 }
 
 spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const float *scores,
@@ -274,8 +291,11 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
         return fail(SPATTN_ERR_UNSUPPORTED, "selection needs %zu bytes of shared memory (max_blocks %d)",
                     smem, a.max_blocks);
     SP_TRY(ensure_smem((const void *)select_kernel, (int)smem));
-    select_kernel<<<d->batch * d->num_kv_heads, kSelThreads, smem, st>>>(a);
-    return cuda_ok(cudaGetLastError(), "select launch");
+    // short rows: fewer threads; from 1024 middle blocks up, a full CTA
+    const int nm = n_mid_cap(d, p);
+    const int threads = nm <= 1024 ? 256 : kSelThreads;
+    return cuda_ok(launch(select_kernel, dim3(d->batch * d->num_kv_heads), dim3(threads), smem, st, a),
+                   "select launch");
 }
 
 std::map<std::pair<int, const void *>, int> g_occ;
@@ -305,9 +325,9 @@ spattn_status launch_attn_t(AttnArgs &a, int sms, cudaStream_t st, int *ctas_out
     int per_sm;
     SP_TRY(resident_ctas(fn, kAttnThreads, smem, attn_ctas_per_sm(RG), &per_sm));
     const int ctas = std::min(kMaxAttnCtas, sms * per_sm);
-    attn_kernel<RG, FP8><<<ctas, kAttnThreads, smem, st>>>(a);
     *ctas_out = ctas;
-    return cuda_ok(cudaGetLastError(), "attention launch");
+    return cuda_ok(launch(attn_kernel<RG, FP8>, dim3(ctas), dim3(kAttnThreads), smem, st, a),
+                   "attention launch");
 }
 
 template <bool FP8>
@@ -373,8 +393,9 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.ctas = ctas;
     const int64_t nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
     const int per = kMergeThreads / 32;
-    merge_kernel<<<(unsigned)((nrows + per - 1) / per), kMergeThreads, 0, st>>>(m);
-    return cuda_ok(cudaGetLastError(), "merge launch");
+    return cuda_ok(launch(merge_kernel, dim3((unsigned)((nrows + per - 1) / per)), dim3(kMergeThreads), 0,
+                              st, m),
+                   "merge launch");
 }
 
 spattn_status check_cache_args(const spattn_dims *d, const void *q, const void *k_cache,
