@@ -49,7 +49,7 @@ struct StageMeta {
     int page;     // page id, -1 when the block or its page is invalid
     int unit;     // b * Hkv + h
     int flags;    // kFirst | kLast | kEnd
-    int unused0;
+    int seg;      // segment id within the CTA (tensor-core kernel)
     int unused1;
     int qslot;    // query slot holding the segment's query rows
     int pad;
@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm(RG)) attn_kerne
         const int64_t lo = W * c / C, hi = W * (c + 1) / C;
         int i_push = 0;  // stages pushed into the ring so far
         int seg = 0;     // segments started so far
+        int qs = 0;      // query slot of the current segment
         // Push one stage (called by the whole warp, uniformly).  At a segment
         // start the warp first writes the unit's query rows, scaled, into
         // query slot seg % kStages: once the stage itself is free, the
@@ -213,8 +214,8 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm(RG)) attn_kerne
             int okw = 1;
             if (lane == 0 && i_push >= kStages) okw = mbar_wait(&empty[s], ((i_push / kStages) - 1) & 1);
             if (!__shfl_sync(0xffffffffu, okw, 0)) return false;
-            const int qs = seg % kStages;
             if (flags & kFirst) {
+                qs = seg % kStages;
                 const int b = unit / a.hkv, h = unit % a.hkv;
                 float *qd = qslots + qs * attn_qslot_floats(RG);
                 for (int task = lane; task < RG * 4 * (kHeadDim / 8); task += 32) {
@@ -515,14 +516,33 @@ struct MergeArgs {
     const int32_t *sel_count;
     float *out;                 // [B][Tq][Hq][D]
     int batch, tq, hq, hkv, group, rows, units, max_sel, ctas;
+    int wslots;                 // partial records per (CTA, unit): 1, or one per tensor-core softmax warp
 };
 
 constexpr int kMergeThreads = 256;
 
+// Record x of a unit's candidate list (CTA c_lo + x / wslots, warp x %
+// wslots), or -1 if it was not written: the CTA's range misses the unit's
+// [pre, pre + cnt) part (only when W < C), or, with one record per
+// tensor-core softmax warp, the warp's pair took none of the CTA's tiles of
+// the unit (pair p takes CTA-local tile indices of parity p).
+__device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int x, int c_lo, int unit, int64_t pre, int cnt,
+                                                int64_t W) {
+    const int cc = c_lo + x / a.wslots, w = x % a.wslots;
+    const int64_t lo_c = W * cc / a.ctas, hi_c = W * (cc + 1) / a.ctas;
+    const int64_t ia = (pre > lo_c ? pre : lo_c) - lo_c;
+    const int64_t ib = (pre + cnt < hi_c ? pre + cnt : hi_c) - lo_c;
+    if (ib <= ia) return -1;
+    if (a.wslots > 1 && ib - ia < 2 && (ia & 1) != (w >> 1)) return -1;
+    return ((int64_t)cc + unit) * a.wslots + w;
+}
+
 // One warp per output row (b, t, query head): out = sum_s 2^(m_s - M) o_s /
-// sum_s 2^(m_s - M) l_s over the segments of the row's unit, i.e. the slots
-// c + unit for the CTAs c whose range meets the unit's part of the sequence.
-// A unit with nothing kept (empty request) gets a zero row.
+// sum_s 2^(m_s - M) l_s over the partial records of the row's unit: slot
+// c + unit for each CTA c whose range meets the unit's part of the sequence
+// (with wslots = 4, record w of that slot for each softmax warp w whose pair
+// took one of the CTA's tiles of the unit: pair w / 2 takes the tiles with
+// CTA-local index of its parity).  A unit with nothing kept gets a zero row.
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t grow = (int64_t)blockIdx.x * (kMergeThreads / 32) + warp;
@@ -548,21 +568,25 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f;
     if (cnt > 0) {
-        // CTAs with an empty range (only when W < C) wrote no partial: skip them
+        // records r = (slot * wslots + w) that were written: CTAs with an
+        // empty range (only when W < C) wrote none; with wslots = 4 a pair
+        // wrote only if it took a tile
         const int c_lo = cta_of(pre, W, a.ctas), c_hi = cta_of(pre + cnt - 1, W, a.ctas);
+        const int nrec = (c_hi - c_lo + 1) * a.wslots;
         float M = -INFINITY;
-        for (int cc = c_lo + lane; cc <= c_hi; cc += 32)
-            if (cta_nonempty(cc, W, a.ctas)) M = fmaxf(M, a.part_ml[(((int64_t)cc + unit) * a.rows + row) * 2]);
+        for (int x = lane; x < nrec; x += 32) {
+            const int64_t r = merge_record(a, x, c_lo, unit, pre, cnt, W);
+            if (r >= 0) M = fmaxf(M, a.part_ml[(r * a.rows + row) * 2]);
+        }
         M = warp_max(M);
         if (M != -INFINITY) {
 #pragma unroll 4
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-                if (!cta_nonempty(cc, W, a.ctas)) continue;
-                const int64_t slot = (int64_t)cc + unit;
-                const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + (slot * a.rows + row) * 2);
+            for (int x = 0; x < nrec; ++x) {
+                const int64_t r = merge_record(a, x, c_lo, unit, pre, cnt, W);
+                if (r < 0) continue;
+                const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
                 const float w = exp2f(ml.x - M);
-                const float4 o =
-                    reinterpret_cast<const float4 *>(a.part_o + (slot * a.rows + row) * kHeadDim)[lane];
+                const float4 o = reinterpret_cast<const float4 *>(a.part_o + (r * a.rows + row) * kHeadDim)[lane];
                 lsum = fmaf(w, ml.y, lsum);
                 acc.x = fmaf(w, o.x, acc.x);
                 acc.y = fmaf(w, o.y, acc.y);

@@ -1,6 +1,7 @@
 // spattn.cu -- C ABI of libspattn: argument checks, workspace layout and
 // kernel launches.  Every kernel lives in the headers included below; this
 // is the only translation unit, so the device status word is one symbol.
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -19,6 +20,7 @@
 #include "scores.cuh"
 #include "select.cuh"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 
 using namespace spattn;
 
@@ -131,6 +133,10 @@ float sm_scale_of(const spattn_params *p) {
 
 int rows_of(const spattn_dims *d) { return d->q_tokens * (d->num_q_heads / d->num_kv_heads); }
 
+// Attention runs on the tensor cores for bf16 caches with at most kTcNQ
+// query rows per KV head, on CUDA cores otherwise.
+bool uses_tc(const spattn_dims *d) { return d->kv_dtype == SPATTN_KV_BF16 && rows_of(d) <= kTcNQ; }
+
 int rg_of(int rows) {
     const int rg = (rows + 3) / 4;
     int p = 1;
@@ -180,12 +186,13 @@ struct DecodeLayout {
     size_t scores_off, scores_bytes, part_o_off, part_ml_off, total;
 };
 
-// Workspace: [scores] | partial outputs | partial (max, sum).  One partial
-// record of `rows` query rows per slot; (C_max + units) slots.
+// Workspace: [scores] | partial outputs | partial (max, sum).  (C_max +
+// units) slots of `rows` query rows, one partial record per slot (CUDA-core
+// kernel) or one per softmax warp (tensor-core kernel, kTcWarpSlots).
 DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
     DecodeLayout L{};
     const int64_t units = (int64_t)d->batch * d->num_kv_heads;
-    const int64_t slots = kMaxAttnCtas + units;
+    const int64_t slots = (kMaxAttnCtas + units) * (uses_tc(d) ? kTcWarpSlots : 1);
     const int64_t rows = rows_of(d);
     size_t off = 0;
     L.scores_off = 0;
@@ -330,6 +337,63 @@ spattn_status launch_attn_t(AttnArgs &a, int sms, cudaStream_t st, int *ctas_out
                    "attention launch");
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// 2-D view of a bf16 cache as [num_pages * Hkv * 64 token rows][128], boxes
+// of 64 x 64 with 128-byte swizzle (the tensor-core operand layout).
+spattn_status kv_tensor_map(CUtensorMap *m, const void *base, int64_t rows) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            SP_TRY(cuda_ok(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q),
+                           "cudaGetDriverEntryPoint"));
+            if (!fn || q != cudaDriverEntryPointSuccess)
+                return fail(SPATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SPATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SPATTN_OK;
+}
+
+// Tensor-core path: bf16 caches, at most kTcNQ query rows per KV head.  One
+// CTA per SM (all of its TMEM), rows rounded up to 4, 8 or 16.
+template <int RQ>
+spattn_status launch_attn_tc_t(AttnArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap, int sms,
+                               cudaStream_t st, int *ctas_out) {
+    const int smem = TcLayout<RQ>::kSmem;
+    const void *fn = (const void *)attn_tc_kernel<RQ>;
+    SP_TRY(ensure_smem(fn, smem));
+    const int ctas = std::min(kMaxAttnCtas, sms);
+    *ctas_out = ctas;
+    return cuda_ok(launch(attn_tc_kernel<RQ>, dim3(ctas), dim3(kTcThreads), smem, st, kmap, vmap, a),
+                   "attention (tensor core) launch");
+}
+
+spattn_status launch_attn_tc(AttnArgs &a, const void *k_cache, const void *v_cache, int sms, cudaStream_t st,
+                             int *ctas_out) {
+    CUtensorMap kmap, vmap;
+    const int64_t rows = (int64_t)a.num_pages * a.hkv * kBlock;
+    SP_TRY(kv_tensor_map(&kmap, k_cache, rows));
+    SP_TRY(kv_tensor_map(&vmap, v_cache, rows));
+    if (a.rows <= 4) return launch_attn_tc_t<4>(a, kmap, vmap, sms, st, ctas_out);
+    if (a.rows <= 8) return launch_attn_tc_t<8>(a, kmap, vmap, sms, st, ctas_out);
+    return launch_attn_tc_t<16>(a, kmap, vmap, sms, st, ctas_out);
+}
+
 template <bool FP8>
 spattn_status launch_attn_rg(int rg, AttnArgs &a, int sms, cudaStream_t st, int *ctas) {
     switch (rg) {
@@ -375,7 +439,11 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     a.max_sel = d->max_sel;
     a.qscale = sm_scale_of(p) * kLog2e;
     int ctas = 0;
-    SP_TRY(fp8 ? launch_attn_rg<true>(rg, a, sms, st, &ctas) : launch_attn_rg<false>(rg, a, sms, st, &ctas));
+    const bool tc = uses_tc(d);
+    if (tc)
+        SP_TRY(launch_attn_tc(a, k_cache, v_cache, sms, st, &ctas));
+    else
+        SP_TRY(fp8 ? launch_attn_rg<true>(rg, a, sms, st, &ctas) : launch_attn_rg<false>(rg, a, sms, st, &ctas));
 
     MergeArgs m;
     m.part_o = a.part_o;
@@ -391,6 +459,7 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.units = a.units;
     m.max_sel = d->max_sel;
     m.ctas = ctas;
+    m.wslots = tc ? kTcWarpSlots : 1;
     const int64_t nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
     const int per = kMergeThreads / 32;
     return cuda_ok(launch(merge_kernel, dim3((unsigned)((nrows + per - 1) / per)), dim3(kMergeThreads), 0,
@@ -444,6 +513,14 @@ spattn_status noalloc_scratch(void **out) {
 static_assert(attn_off_pbuf(false, 1) % 16 == 0 && attn_off_pbuf(true, 16) % 16 == 0, "layout");
 static_assert(2 * (attn_smem_bytes(false, 1) + 1024) <= 228 * 1024, "two CTAs per SM at one row group");
 static_assert(attn_smem_bytes(false, 16) <= 227 * 1024, "one CTA per SM at sixteen row groups");
+template <int RQ>
+constexpr bool tc_layout_ok() {
+    using TL = TcLayout<RQ>;
+    return TL::kSmem <= 227 * 1024 && TL::kStages % 2 == 0 && TL::kOffQ % 1024 == 0 && TL::kQSlot % 1024 == 0 &&
+           TL::kOffP % 1024 == 0 && TL::kOffRing % 1024 == 0 && kTcBox % 1024 == 0 && TL::kOffP >= TL::kOffQ + 1024;
+}
+static_assert(tc_layout_ok<4>() && tc_layout_ok<8>() && tc_layout_ok<16>(),
+              "one CTA per SM; even stage count; swizzled operand tiles on 1024-byte boundaries");
 
 }  // namespace
 
