@@ -16,7 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libspattn.so")
 SOURCES = ["spattn.cu"]
-DEPS = ["common.cuh", "compress.cuh", "scores.cuh", "select.cuh", "attention.cuh", "exports.map"]
+DEPS = ["common.cuh", "compress.cuh", "scores.cuh", "select.cuh", "attention.cuh", "tcgen05.cuh",
+        "attention_tc.cuh", "exports.map"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
