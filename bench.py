@@ -44,7 +44,7 @@ from block_sparse_kv_spattn_b200.workloads import BENCH_WORKLOAD, WORKLOADS, mak
 METRIC = "selected-KV HBM GB/s (% of ~8 TB/s) and decode queries/s at 128K ctx, 1 B200"
 FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
-ATTN_SOURCES = ["common.cuh", "attention.cuh"]
+ATTN_SOURCES = ["common.cuh", "attention.cuh", "tcgen05.cuh", "attention_tc.cuh"]
 
 
 def _peaks():
@@ -62,6 +62,15 @@ def attn_source_hash() -> str:
         with open(os.path.join(ROOT, "block_sparse_kv_spattn_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def attn_label(w) -> str:
+    """The attention kernels one decode_selected call launches (timed together)."""
+    rows = w.q_tokens * (w.num_q_heads // w.num_kv_heads)
+    if not w.kv_fp8 and rows <= 16:
+        rq = 4 if rows <= 4 else (8 if rows <= 8 else 16)
+        return f"attention (attn_tc_kernel<{rq}> on tcgen05 + merge_kernel, one decode_selected call)"
+    return "attention (attn_kernel + merge_kernel, one decode_selected call)"
 
 
 def measured_traffic(units_in_launch: float):
@@ -302,7 +311,7 @@ def run_native(args, rank, world, local_rank):
         "hbm_fraction": round(value / peak, 4),
         "queries_per_s": round(queries, 1),
         "bytes_per_step": bts,
-        "roofline": {"kernel": "attention (attn_kernel + merge_kernel, one decode_selected call)",
+        "roofline": {"kernel": attn_label(w),
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                      "unit": "GB/s", "frac": round(achieved / peak, 4),

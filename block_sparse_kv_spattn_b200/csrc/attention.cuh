@@ -519,7 +519,7 @@ struct MergeArgs {
     int wslots;                 // partial records per (CTA, unit): 1, or one per tensor-core softmax warp
 };
 
-constexpr int kMergeThreads = 256;
+constexpr int kMergeThreads = 64;   // small CTAs: the rows spread over many SMs
 
 // Record x of a unit's candidate list (CTA c_lo + x / wslots, warp x %
 // wslots), or -1 if it was not written: the CTA's range misses the unit's
@@ -573,6 +573,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
         // wrote only if it took a tile
         const int c_lo = cta_of(pre, W, a.ctas), c_hi = cta_of(pre + cnt - 1, W, a.ctas);
         const int nrec = (c_hi - c_lo + 1) * a.wslots;
+        // (m, l) of the records, 32 at a time across the lanes
         float M = -INFINITY;
         for (int x = lane; x < nrec; x += 32) {
             const int64_t r = merge_record(a, x, c_lo, unit, pre, cnt, W);
@@ -580,19 +581,29 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
         }
         M = warp_max(M);
         if (M != -INFINITY) {
-#pragma unroll 4
-            for (int x = 0; x < nrec; ++x) {
-                const int64_t r = merge_record(a, x, c_lo, unit, pre, cnt, W);
-                if (r < 0) continue;
-                const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
-                const float w = exp2f(ml.x - M);
-                const float4 o = reinterpret_cast<const float4 *>(a.part_o + (r * a.rows + row) * kHeadDim)[lane];
-                lsum = fmaf(w, ml.y, lsum);
-                acc.x = fmaf(w, o.x, acc.x);
-                acc.y = fmaf(w, o.y, acc.y);
-                acc.z = fmaf(w, o.z, acc.z);
-                acc.w = fmaf(w, o.w, acc.w);
+            for (int x0 = 0; x0 < nrec; x0 += 32) {
+                // lane e holds record x0 + e: its index and weight 2^(m - M)
+                const int64_t r = x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
+                float w = 0.f;
+                if (r >= 0) {
+                    const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
+                    w = exp2f(ml.x - M);
+                    lsum = fmaf(w, ml.y, lsum);
+                }
+                const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
+#pragma unroll 8
+                for (int e = 0; e < n_here; ++e) {
+                    const float we = __shfl_sync(0xffffffffu, w, e);
+                    const int64_t re = __shfl_sync(0xffffffffu, r, e);
+                    if (re < 0 || we == 0.f) continue;   // uniform
+                    const float4 o = reinterpret_cast<const float4 *>(a.part_o + (re * a.rows + row) * kHeadDim)[lane];
+                    acc.x = fmaf(we, o.x, acc.x);
+                    acc.y = fmaf(we, o.y, acc.y);
+                    acc.z = fmaf(we, o.z, acc.z);
+                    acc.w = fmaf(we, o.w, acc.w);
+                }
             }
+            lsum = warp_sum(lsum);
         }
     }
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;

@@ -287,18 +287,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int nb = (L + kBlock - 1) / kBlock;
                 for (int i0 = ia; i0 < ib && ok; i0 += 32) {
                     // lane l resolves tile i0 + l: block index and page, checked
+                    // (the table load does not wait for the length check)
                     int jl = 0, pl = -1;
                     if (i0 + lane < ib) {
                         jl = sel[i0 + lane];
-                        if (jl >= 0 && jl < nb) {
-                            const int pg = a.block_table[(int64_t)b * a.max_blocks + jl];
-                            if (pg >= 0 && pg < a.num_pages)
-                                pl = pg;
-                            else
-                                flag(SPATTN_DEV_BAD_PAGE);
-                        } else {
+                        const bool in_table = jl >= 0 && jl < a.max_blocks;
+                        const int pg = in_table ? a.block_table[(int64_t)b * a.max_blocks + jl] : -1;
+                        if (!in_table || jl >= nb)
                             flag(SPATTN_DEV_BAD_BLOCK);
-                        }
+                        else if (pg < 0 || pg >= a.num_pages)
+                            flag(SPATTN_DEV_BAD_PAGE);
+                        else
+                            pl = pg;
                     }
                     const int n_here = ib - i0 < 32 ? ib - i0 : 32;
                     for (int e = 0; e < n_here && ok; ++e) {
