@@ -59,7 +59,8 @@ __host__ __device__ inline size_t select_smem_bytes(int n_mid_cap, int sort_cap,
 
 // ------------------------------------------------------------ block helpers
 
-// Block-wide max and min of one uint32 per thread (every thread calls it).
+// Block-wide max and min of one uint32 per thread (every thread calls it):
+// per-warp reductions, then every warp reduces the warps' results.
 __device__ __forceinline__ void block_minmax_u32(uint32_t vmax, uint32_t vmin, int *tmp, uint32_t &omax,
                                                  uint32_t &omin) {
     vmax = __reduce_max_sync(0xffffffffu, vmax);
@@ -70,23 +71,21 @@ __device__ __forceinline__ void block_minmax_u32(uint32_t vmax, uint32_t vmin, i
         tmp[32 + (threadIdx.x >> 5)] = (int)vmin;
     }
     __syncthreads();
-    omax = 0;
-    omin = 0xffffffffu;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-        omax = max(omax, (uint32_t)tmp[w]);
-        omin = min(omin, (uint32_t)tmp[32 + w]);
-    }
+    const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    omax = __reduce_max_sync(0xffffffffu, lane < nw ? (uint32_t)tmp[lane] : 0u);
+    omin = __reduce_min_sync(0xffffffffu, lane < nw ? (uint32_t)tmp[32 + lane] : 0xffffffffu);
 }
 
-// Block-wide sum of one float per thread, added in a fixed order.
+// Block-wide sum of one float per thread: per-warp butterflies, then a
+// butterfly over the warps' sums (the same fixed order on every run; every
+// lane ends with the same bits).
 __device__ __forceinline__ float block_sum_f(float v, float *tmp) {
     v = warp_sum(v);
     __syncthreads();
     if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = v;
     __syncthreads();
-    float r = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += tmp[w];
-    return r;
+    const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    return warp_sum(lane < nw ? tmp[lane] : 0.f);
 }
 
 // Middle scores of a row -> order-preserving keys in shared memory.  The
@@ -229,6 +228,7 @@ __device__ Cut find_cut(const SelectShared &sh, int n, int k, uint32_t kmax, uin
                 const uint32_t kt = sh.cand_key[t];
                 const int it = sh.cand_idx[t];
                 int rank = 0;
+#pragma unroll 8
                 for (int u = 0; u < c; ++u) {
                     const uint32_t ku = sh.cand_key[u];
                     rank += ku > kt || (ku == kt && sh.cand_idx[u] < it);
@@ -322,6 +322,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     }
     const int bh = blockIdx.x;
     const int b = bh / a.hkv, h = bh % a.hkv;
+    // the first token's score row into L1 while the length is fetched
+    {
+        const float *row0 = a.scores + ((int64_t)b * a.tq * a.hkv + h) * a.max_blocks;
+        for (int i = threadIdx.x * 32; i < a.n_mid_cap + a.sink; i += blockDim.x * 32)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(row0 + i));
+    }
     int L = a.seq_lens[b];
     if (L < 0 || L > a.max_blocks * kBlock) {
         if (threadIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
