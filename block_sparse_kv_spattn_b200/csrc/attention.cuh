@@ -573,38 +573,47 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
         // wrote only if it took a tile
         const int c_lo = cta_of(pre, W, a.ctas), c_hi = cta_of(pre + cnt - 1, W, a.ctas);
         const int nrec = (c_hi - c_lo + 1) * a.wslots;
-        // (m, l) of the records, 32 at a time across the lanes
+        // batches of 32 records, one per lane, merged online: the lanes load
+        // their records' (m, l) together, then the row's O of every record of
+        // the batch is loaded in one unrolled run (no record waits on another)
         float M = -INFINITY;
-        for (int x = lane; x < nrec; x += 32) {
-            const int64_t r = merge_record(a, x, c_lo, unit, pre, cnt, W);
-            if (r >= 0) M = fmaxf(M, a.part_ml[(r * a.rows + row) * 2]);
-        }
-        M = warp_max(M);
-        if (M != -INFINITY) {
-            for (int x0 = 0; x0 < nrec; x0 += 32) {
-                // lane e holds record x0 + e: its index and weight 2^(m - M)
-                const int64_t r = x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
-                float w = 0.f;
-                if (r >= 0) {
-                    const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
-                    w = exp2f(ml.x - M);
-                    lsum = fmaf(w, ml.y, lsum);
-                }
-                const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
-#pragma unroll 8
-                for (int e = 0; e < n_here; ++e) {
-                    const float we = __shfl_sync(0xffffffffu, w, e);
-                    const int64_t re = __shfl_sync(0xffffffffu, r, e);
-                    if (re < 0 || we == 0.f) continue;   // uniform
-                    const float4 o = reinterpret_cast<const float4 *>(a.part_o + (re * a.rows + row) * kHeadDim)[lane];
-                    acc.x = fmaf(we, o.x, acc.x);
-                    acc.y = fmaf(we, o.y, acc.y);
-                    acc.z = fmaf(we, o.z, acc.z);
-                    acc.w = fmaf(we, o.w, acc.w);
-                }
+        for (int x0 = 0; x0 < nrec; x0 += 32) {
+            const int64_t r = x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
+            float2 ml = make_float2(-INFINITY, 0.f);
+            if (r >= 0) ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
+            const float Mb = fmaxf(M, warp_max(ml.x));
+            const unsigned valid = __ballot_sync(0xffffffffu, r >= 0 && ml.x != -INFINITY);
+            if (Mb == -INFINITY || !valid) continue;   // uniform: nothing to add
+            if (Mb != M) {   // uniform: rescale what is summed so far
+                const float f = M == -INFINITY ? 0.f : exp2f(M - Mb);
+                acc.x *= f;
+                acc.y *= f;
+                acc.z *= f;
+                acc.w *= f;
+                lsum *= f;
+                M = Mb;
             }
-            lsum = warp_sum(lsum);
+            float w = 0.f;
+            if ((valid >> lane) & 1u) {
+                w = exp2f(ml.x - M);
+                lsum = fmaf(w, ml.y, lsum);
+            }
+            // records without weight read the first valid one (weight 0)
+            const int64_t rfirst = __shfl_sync(0xffffffffu, r, __ffs(valid) - 1);
+            const int64_t rr = ((valid >> lane) & 1u) ? r : rfirst;
+            const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
+#pragma unroll 16
+            for (int e = 0; e < n_here; ++e) {
+                const float we = __shfl_sync(0xffffffffu, w, e);
+                const int64_t re = __shfl_sync(0xffffffffu, rr, e);
+                const float4 o = reinterpret_cast<const float4 *>(a.part_o + (re * a.rows + row) * kHeadDim)[lane];
+                acc.x = fmaf(we, o.x, acc.x);
+                acc.y = fmaf(we, o.y, acc.y);
+                acc.z = fmaf(we, o.z, acc.z);
+                acc.w = fmaf(we, o.w, acc.w);
+            }
         }
+        lsum = warp_sum(lsum);
     }
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
     reinterpret_cast<float4 *>(a.out + grow * kHeadDim)[lane] =
