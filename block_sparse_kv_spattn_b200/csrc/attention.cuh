@@ -519,7 +519,7 @@ struct MergeArgs {
     int wslots;                 // partial records per (CTA, unit): 1, or one per tensor-core softmax warp
 };
 
-constexpr int kMergeThreads = 64;   // small CTAs: the rows spread over many SMs
+constexpr int kMergeMaxWarps = 8;   // warps per output row, for units split over many CTAs
 
 // Record x of a unit's candidate list (CTA c_lo + x / wslots, warp x %
 // wslots), or -1 if it was not written: the CTA's range misses the unit's
@@ -537,16 +537,19 @@ __device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int x, int c
     return ((int64_t)cc + unit) * a.wslots + w;
 }
 
-// One warp per output row (b, t, query head): out = sum_s 2^(m_s - M) o_s /
+// One CTA per output row (b, t, query head): out = sum_s 2^(m_s - M) o_s /
 // sum_s 2^(m_s - M) l_s over the partial records of the row's unit: slot
 // c + unit for each CTA c whose range meets the unit's part of the sequence
 // (with wslots = 4, record w of that slot for each softmax warp w whose pair
 // took one of the CTA's tiles of the unit: pair w / 2 takes the tiles with
-// CTA-local index of its parity).  A unit with nothing kept gets a zero row.
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t grow = (int64_t)blockIdx.x * (kMergeThreads / 32) + warp;
-    if (grow >= (int64_t)a.batch * a.tq * a.hq) return;
+// CTA-local index of its parity).  The CTA's warps take batches of 32
+// records in turn (a unit split over many CTAs has hundreds) and are
+// combined through shared memory.  A unit with nothing kept gets a zero row.
+__global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a) {
+    __shared__ float s_m[kMergeMaxWarps], s_l[kMergeMaxWarps];
+    __shared__ float4 s_acc[kMergeMaxWarps][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int64_t grow = blockIdx.x;
     const int i = (int)(grow % a.hq);
     const int t = (int)((grow / a.hq) % a.tq);
     const int b = (int)(grow / ((int64_t)a.hq * a.tq));
@@ -566,7 +569,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
     }
     const int cnt = min(max(a.sel_count[unit], 0), a.max_sel);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lsum = 0.f;
+    float lsum = 0.f, M = -INFINITY;
     if (cnt > 0) {
         // records r = (slot * wslots + w) that were written: CTAs with an
         // empty range (only when W < C) wrote none; with wslots = 4 a pair
@@ -576,8 +579,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
         // batches of 32 records, one per lane, merged online: the lanes load
         // their records' (m, l) together, then the row's O of every record of
         // the batch is loaded in one unrolled run (no record waits on another)
-        float M = -INFINITY;
-        for (int x0 = 0; x0 < nrec; x0 += 32) {
+        for (int x0 = 32 * warp; x0 < nrec; x0 += 32 * nw) {
             const int64_t r = x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
             float2 ml = make_float2(-INFINITY, 0.f);
             if (r >= 0) ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
@@ -614,6 +616,31 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeArgs a) {
             }
         }
         lsum = warp_sum(lsum);
+    }
+    if (nw > 1) {
+        // combine the warps: weights 2^(M_w - M)
+        if (lane == 0) {
+            s_m[warp] = M;
+            s_l[warp] = lsum;
+        }
+        s_acc[warp][lane] = acc;
+        __syncthreads();
+        if (warp != 0) return;
+        float Mt = -INFINITY;
+        for (int w = 0; w < nw; ++w) Mt = fmaxf(Mt, s_m[w]);
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        lsum = 0.f;
+        if (Mt != -INFINITY)
+            for (int w = 0; w < nw; ++w) {
+                if (s_m[w] == -INFINITY) continue;
+                const float f = exp2f(s_m[w] - Mt);
+                const float4 o = s_acc[w][lane];
+                lsum = fmaf(f, s_l[w], lsum);
+                acc.x = fmaf(f, o.x, acc.x);
+                acc.y = fmaf(f, o.y, acc.y);
+                acc.z = fmaf(f, o.z, acc.z);
+                acc.w = fmaf(f, o.w, acc.w);
+            }
     }
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
     reinterpret_cast<float4 *>(a.out + grow * kHeadDim)[lane] =

@@ -461,11 +461,13 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.max_sel = d->max_sel;
     m.ctas = ctas;
     m.wslots = tc ? kTcWarpSlots : 1;
+    // one CTA per output row; warps for the records a unit gets on average
+    // (CTAs per unit + 1, times the records per CTA), 32 per warp
     const int64_t nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
-    const int per = kMergeThreads / 32;
-    return cuda_ok(launch(merge_kernel, dim3((unsigned)((nrows + per - 1) / per)), dim3(kMergeThreads), 0,
-                              st, m),
-                   "merge launch");
+    const int64_t recs = ((int64_t)ctas / std::max(1, a.units) + 2) * m.wslots;
+    int wpr = 1;
+    while (wpr < kMergeMaxWarps && 32 * wpr < recs) wpr *= 2;
+    return cuda_ok(launch(merge_kernel, dim3((unsigned)nrows), dim3(32 * wpr), 0, st, m), "merge launch");
 }
 
 spattn_status check_cache_args(const spattn_dims *d, const void *q, const void *k_cache,
