@@ -178,7 +178,7 @@ def run_native(args, rank, world, local_rank):
     q, kc, vc, ks, vs = inp["q"], inp["k_cache"], inp["v_cache"], inp["k_scale"], inp["v_scale"]
     bt, sl = inp["block_table"], inp["seq_lens"]
     params = spattn.Params(sink_blocks=w.sink_blocks, local_blocks=w.local_blocks, mode=w.mode,
-                           top_k=w.top_k, top_p=w.top_p, max_ratio=w.max_ratio)
+                           top_k=w.top_k, top_p=w.top_p, max_ratio=w.max_ratio, min_ratio=w.min_ratio)
     dims = spattn.dims_for(q, kc, bt)
     max_sel = spattn.required_max_sel(dims, params)
     dims.max_sel = max_sel
@@ -206,14 +206,21 @@ def run_native(args, rank, world, local_rank):
     assert Tq <= (w.local_blocks - 1) * w.block_size + 1, "append would touch a middle block"
     side = torch.cuda.Stream()
 
+    anchored = w.mode == "topp_anchor"   # the local blocks are scored: compress first
+
     def front():   # scores + selection, with the tail block's compression beside them
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
+        if anchored:
             spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
                                  q_tokens=Tq)
+        else:
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
+                                     q_tokens=Tq)
         spattn.block_scores(q, kbar, bt, sl, scores, params, k_cache=kc)
         spattn.select(scores, sl, sel_idx, sel_count, params, q=q, k_cache=kc, block_table=bt)
-        torch.cuda.current_stream().wait_stream(side)
+        if not anchored:
+            torch.cuda.current_stream().wait_stream(side)
 
     def attend():  # sparse attention + split merge
         spattn.decode_selected(q, kc, vc, ks, vs, bt, sl, sel_idx, sel_count, out, ws, params)
@@ -312,8 +319,9 @@ def run_native(args, rank, world, local_rank):
         "config": {"workload": w.name, "batch": B, "q_tokens": Tq, "num_q_heads": w.num_q_heads,
                    "num_kv_heads": Hkv, "seq_len": w.seq_len, "block": w.block_size,
                    "sink_blocks": w.sink_blocks, "local_blocks": w.local_blocks,
-                   "selection": f"{w.mode} p={w.top_p} cap={w.max_ratio}" if w.mode == "topp" else
-                   f"{w.mode} k={w.top_k} ratio={w.max_ratio}",
+                   "selection": (f"{w.mode} p={w.top_p} cap={w.max_ratio}" if w.mode == "topp" else
+                                 f"{w.mode} p={w.top_p} cap={w.min_ratio}-{w.max_ratio} by anchors"
+                                 if w.mode == "topp_anchor" else f"{w.mode} k={w.top_k} ratio={w.max_ratio}"),
                    "l2": "flushed between steps (512 MB write, then a 512 MB read so the flush's dirty lines are written back; outside the timed events)",
                    "parallelism": f"independent replicas x{world}"},
         "hbm_fraction": round(value / peak, 4),

@@ -19,6 +19,7 @@ struct ScoresArgs {
     const int32_t *seq_lens;
     float *scores;            // [B][Tq][Hkv][max_blocks]
     int tq, hq, num_pages, max_blocks, sink, local, bpc;
+    int anchors;              // also score the sink and local blocks (anchor-adaptive selection)
     float scale;
 };
 
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     for (int jj = threadIdx.x; jj < a.bpc; jj += kScoreThreads) {
         const int j = j0 + jj;
         int page = -1;
-        if (j < a.max_blocks && j >= a.sink && j < nb - a.local) {
+        if (j < a.max_blocks && j < nb && (a.anchors || (j >= a.sink && j < nb - a.local))) {
             page = a.block_table[(int64_t)b * a.max_blocks + j];
             if (page < 0 || page >= a.num_pages) {
                 flag(SPATTN_DEV_BAD_PAGE);

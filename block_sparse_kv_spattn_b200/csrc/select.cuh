@@ -26,7 +26,7 @@ struct SelectArgs {
     int32_t *sel_idx;          // [B][Hkv][max_sel]
     int32_t *sel_count;        // [B][Hkv]
     int tq, hkv, max_blocks, max_sel, sink, local, mode, top_k;
-    float top_p, max_ratio;
+    float top_p, max_ratio, min_ratio;
     int n_mid_cap;             // keys capacity (>= every row's middle count)
     int sort_cap;              // power-of-two sort capacity (top-p), else 0
 };
@@ -346,8 +346,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
 
     for (int t = 0; t < a.tq && n_mid > 0; ++t) {
         const float *row = a.scores + (((int64_t)b * a.tq + t) * a.hkv + h) * a.max_blocks + S;
-        const int k = a.mode == SPATTN_SEL_TOPK ? k_topk : k_max;
-        if (k <= 0) continue;
+        const bool anchor = a.mode == SPATTN_SEL_TOPP_ANCHOR;
+        int k = a.mode == SPATTN_SEL_TOPK ? k_topk : k_max;
+        if (k <= 0 && !anchor) continue;
         if (a.mode == SPATTN_SEL_TOPK && k >= n_mid) {
             for (int i = threadIdx.x; i < n_mid; i += blockDim.x) sh.flags[S + i] = 1;
             __syncthreads();
@@ -356,6 +357,23 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         uint32_t kmax_l, kmin_l, kmax, kmin;
         load_keys(sh, row, a.n_mid_cap, &n_mid, kmax_l, kmin_l);
         block_minmax_u32(kmax_l, kmin_l, sh.itmp, kmax, kmin);
+        if (anchor) {
+            // cap from the anchors: a = their best score, hi / lo the middle's
+            // extremes; r = clamp((hi - a) / (hi - lo), 0, 1), ratio = min_ratio
+            // + r * (max_ratio - min_ratio), k = floor(ratio * n_mid), all in
+            // double with separately rounded operations
+            const float *full = row - S;
+            float amax = -INFINITY;
+            for (int j = 0; j < S; ++j) amax = fmaxf(amax, full[j]);       // n_mid > 0: nb > S + W
+            for (int j = nb - W; j < nb; ++j) amax = fmaxf(amax, full[j]);
+            const double hi = (double)key_float(kmax), lo = (double)key_float(kmin);
+            double r = hi > lo ? __ddiv_rn(__dsub_rn(hi, (double)amax), __dsub_rn(hi, lo)) : 0.0;
+            r = r < 0.0 ? 0.0 : (r > 1.0 ? 1.0 : r);
+            const double ratio =
+                __dadd_rn((double)a.min_ratio, __dmul_rn(r, __dsub_rn((double)a.max_ratio, (double)a.min_ratio)));
+            k = min(n_mid, (int)floor(__dmul_rn(ratio, (double)n_mid)));
+            if (k <= 0) continue;
+        }
         if (a.mode == SPATTN_SEL_TOPK) {
             const Cut cut = find_cut(sh, n_mid, k, kmax, kmin);
             for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });

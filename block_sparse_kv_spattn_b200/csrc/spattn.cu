@@ -92,15 +92,19 @@ spattn_status check_params(const spattn_params *p) {
     if (!p) return fail(SPATTN_ERR_INVALID_ARG, "params is NULL");
     if (p->sink_blocks < 0 || p->local_blocks < 0)
         return fail(SPATTN_ERR_INVALID_ARG, "sink_blocks and local_blocks must be >= 0");
-    if (p->mode != SPATTN_SEL_TOPK && p->mode != SPATTN_SEL_TOPP)
+    if (p->mode != SPATTN_SEL_TOPK && p->mode != SPATTN_SEL_TOPP && p->mode != SPATTN_SEL_TOPP_ANCHOR)
         return fail(SPATTN_ERR_INVALID_ARG, "mode %d", p->mode);
     if (p->top_k < 0) return fail(SPATTN_ERR_INVALID_ARG, "top_k %d < 0", p->top_k);
-    if (p->mode == SPATTN_SEL_TOPP && !(p->top_p > 0.f && p->top_p <= 1.f))
+    if (p->mode != SPATTN_SEL_TOPK && !(p->top_p > 0.f && p->top_p <= 1.f))
         return fail(SPATTN_ERR_INVALID_ARG, "top_p %g not in (0, 1]", (double)p->top_p);
     if (!(p->max_ratio >= 0.f && p->max_ratio <= 1.f))
         return fail(SPATTN_ERR_INVALID_ARG, "max_ratio %g not in [0, 1]", (double)p->max_ratio);
     if (!(p->sm_scale >= 0.f) || !std::isfinite(p->sm_scale))
         return fail(SPATTN_ERR_INVALID_ARG, "sm_scale %g", (double)p->sm_scale);
+    if (p->mode == SPATTN_SEL_TOPP_ANCHOR &&
+        !(p->max_ratio > 0.f && p->min_ratio >= 0.f && p->min_ratio <= p->max_ratio))
+        return fail(SPATTN_ERR_INVALID_ARG, "anchor mode needs 0 <= min_ratio (%g) <= max_ratio (%g), max_ratio > 0",
+                    (double)p->min_ratio, (double)p->max_ratio);
     return SPATTN_OK;
 }
 
@@ -241,6 +245,7 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     a.max_blocks = d->max_blocks_per_seq;
     a.sink = p->sink_blocks;
     a.local = p->local_blocks;
+    a.anchors = p->mode == SPATTN_SEL_TOPP_ANCHOR;
     a.scale = sm_scale_of(p);
     const int rowsq = d->q_tokens * d->num_kv_heads;
     a.bpc = score_blocks_per_cta(rowsq);
@@ -282,12 +287,13 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
     a.sink = p->sink_blocks;
     a.local = p->local_blocks;
     a.mode = p->mode;
+    a.min_ratio = p->min_ratio;
     a.top_k = p->top_k;
     a.top_p = p->top_p;
     a.max_ratio = p->max_ratio;
     a.n_mid_cap = std::max(1, n_mid_cap(d, p));
     a.sort_cap = 0;
-    if (p->mode == SPATTN_SEL_TOPP) {
+    if (p->mode != SPATTN_SEL_TOPK) {
         const int km = std::max(1, k_max_of(p, n_mid_cap(d, p)));
         int np2 = 1;
         while (np2 < km) np2 <<= 1;

@@ -29,7 +29,8 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORK
                 5: "TIMEOUT", 6: "DEVICE"}
 DEV_BAD_PAGE, DEV_BAD_BLOCK, DEV_SEL_OVERFLOW, DEV_WAIT_TIMEOUT, DEV_BAD_LEN = 1, 2, 4, 8, 16
 KV_BF16, KV_FP8_E4M3 = 0, 1
-SEL_TOPK, SEL_TOPP = 0, 1
+SEL_TOPK, SEL_TOPP, SEL_TOPP_ANCHOR = 0, 1, 2
+SEL_MODES = {"topk": SEL_TOPK, "topp": SEL_TOPP, "topp_anchor": SEL_TOPP_ANCHOR}
 
 EXPORTS = ("spattn_required_max_sel", "spattn_compress_keys", "spattn_block_scores",
            "spattn_select", "spattn_decode_workspace_size", "spattn_decode_selected",
@@ -52,7 +53,7 @@ class CDims(ctypes.Structure):
 class CParams(ctypes.Structure):
     _fields_ = [("sink_blocks", ctypes.c_int32), ("local_blocks", ctypes.c_int32),
                 ("mode", ctypes.c_int32), ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float),
-                ("max_ratio", ctypes.c_float), ("sm_scale", ctypes.c_float)]
+                ("max_ratio", ctypes.c_float), ("sm_scale", ctypes.c_float), ("min_ratio", ctypes.c_float)]
 
 
 @dataclasses.dataclass
@@ -60,15 +61,16 @@ class Params:
     """Selection parameters (spattn_params)."""
     sink_blocks: int = 1
     local_blocks: int = 2
-    mode: str = "topk"      # "topk" | "topp"
+    mode: str = "topk"      # "topk" | "topp" | "topp_anchor"
     top_k: int = 0
     top_p: float = 1.0
     max_ratio: float = 0.0
     sm_scale: float = 0.0
+    min_ratio: float = 0.0  # topp_anchor: the cap ratio when the anchors dominate
 
     def c(self) -> CParams:
-        return CParams(self.sink_blocks, self.local_blocks, SEL_TOPK if self.mode == "topk" else SEL_TOPP,
-                       self.top_k, self.top_p, self.max_ratio, self.sm_scale)
+        return CParams(self.sink_blocks, self.local_blocks, SEL_MODES[self.mode],
+                       self.top_k, self.top_p, self.max_ratio, self.sm_scale, self.min_ratio)
 
 
 _lib = None

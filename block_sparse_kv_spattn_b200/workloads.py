@@ -49,10 +49,11 @@ class Workload:
     structure: str = "zipf"           # "zipf" | "planted" | "none"
     n_planted: int = 0
     contiguous: bool = False
-    mode: str = "topp"                # "topk" | "topp"
+    mode: str = "topp"                # "topk" | "topp" | "topp_anchor"
     top_k: int = 0
     top_p: float = 1.0
     max_ratio: float = 0.0
+    min_ratio: float = 0.0            # topp_anchor: the cap ratio when the anchors dominate
     sink_blocks: int = 1
     local_blocks: int = 2
     head_dim: int = HEAD_DIM
@@ -74,6 +75,13 @@ WORKLOADS = {
     "decode_128k_b8": Workload("decode_128k_b8", batch=8, q_tokens=1, num_q_heads=32, num_kv_heads=8,
                                seq_len=131072, structure="zipf", mode="topp", top_p=0.9,
                                max_ratio=0.15, seed=1236),
+    # the gate shape with the anchor-adaptive cap: ratio between 10 % and 20 %
+    # of the middle blocks by how far the best middle block stands above the
+    # sink and local blocks
+    "decode_128k_b8_anchor": Workload("decode_128k_b8_anchor", batch=8, q_tokens=1, num_q_heads=32,
+                                      num_kv_heads=8, seq_len=131072, structure="zipf",
+                                      mode="topp_anchor", top_p=0.9, min_ratio=0.10, max_ratio=0.20,
+                                      seed=1241),
     # the same shape with 2 requests: small enough for detailed profiling
     "decode_128k_b2": Workload("decode_128k_b2", batch=2, q_tokens=1, num_q_heads=32, num_kv_heads=8,
                                seq_len=131072, structure="zipf", mode="topp", top_p=0.9,

@@ -89,7 +89,21 @@ typedef enum {
 #define SPATTN_DEV_BAD_LEN       0x10  /* seq_len < 0 or > max_blocks_per_seq * P */
 
 typedef enum { SPATTN_KV_BF16 = 0, SPATTN_KV_FP8_E4M3 = 1 } spattn_kv_dtype;
-typedef enum { SPATTN_SEL_TOPK = 0, SPATTN_SEL_TOPP = 1 } spattn_sel_mode;
+/*
+ * Selection modes.  SPATTN_SEL_TOPP_ANCHOR: top-p whose retention cap adapts
+ * to the anchors ("Claude Opus 长上下文 KV Cache 稀疏注意力", §多上下文场景下的跨文档
+ * 注意力恢复, anchor-based dynamic selection: the sink and local blocks are
+ * the anchors; the bounds (max, min) of the scores set the Top-P ratio, more
+ * when the maximum stands well above the anchors, less otherwise).  Reading
+ * taken (the page gives no formula): with a = the anchors' highest score and
+ * hi / lo the middle blocks' highest / lowest score of the query row,
+ * r = clamp((hi - a) / (hi - lo), 0, 1) (0 when hi <= lo), ratio = min_ratio
+ * + r * (max_ratio - min_ratio), k_max = floor(ratio * n_mid) (computed in
+ * double from the fp32 scores), then top-p with that cap.  block_scores then
+ * scores the anchor blocks too (so the local blocks' compressed keys must be
+ * current before it runs).
+ */
+typedef enum { SPATTN_SEL_TOPK = 0, SPATTN_SEL_TOPP = 1, SPATTN_SEL_TOPP_ANCHOR = 2 } spattn_sel_mode;
 
 typedef struct {
     int32_t batch;              /* B >= 1 */
@@ -113,6 +127,8 @@ typedef struct {
     float max_ratio;            /* cap k_max = floor(max_ratio * n_mid), in
                                    [0, 1]; 0 means no cap (k_max = n_mid) */
     float sm_scale;             /* softmax and score scale; 0 = 1/sqrt(d) */
+    float min_ratio;            /* SPATTN_SEL_TOPP_ANCHOR: ratio when the anchors
+                                   dominate, in [0, max_ratio] (other modes ignore it) */
 } spattn_params;
 
 /*

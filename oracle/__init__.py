@@ -32,7 +32,7 @@ class _Params(ctypes.Structure):
     _fields_ = [("sink_blocks", ctypes.c_int), ("local_blocks", ctypes.c_int),
                 ("mode", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("top_p", ctypes.c_double), ("max_ratio", ctypes.c_double),
-                ("sm_scale", ctypes.c_double)]
+                ("sm_scale", ctypes.c_double), ("min_ratio", ctypes.c_double)]
 
 
 @dataclasses.dataclass
@@ -58,16 +58,18 @@ class Dims:
 class Params:
     sink_blocks: int = 1
     local_blocks: int = 2
-    mode: str = "topk"          # "topk" | "topp"
+    mode: str = "topk"          # "topk" | "topp" | "topp_anchor"
     top_k: int = 0
     top_p: float = 1.0
     max_ratio: float = 0.0
     sm_scale: float = 0.0
+    min_ratio: float = 0.0      # topp_anchor: the cap ratio when the anchors dominate
 
     def c(self) -> _Params:
         return _Params(self.sink_blocks, self.local_blocks,
-                       0 if self.mode == "topk" else 1, self.top_k,
-                       float(self.top_p), float(self.max_ratio), float(self.sm_scale))
+                       {"topk": 0, "topp": 1, "topp_anchor": 2}[self.mode], self.top_k,
+                       float(self.top_p), float(self.max_ratio), float(self.sm_scale),
+                       float(self.min_ratio))
 
 
 def lib():

@@ -20,7 +20,7 @@ def build(force: bool = False) -> str:
     # -O2 without fast-math: IEEE semantics (NaN, -inf, exact comparisons) are
     # part of the definition.  OpenMP parallelises over independent
     # (request, head) units only; a compiler without it builds a serial oracle.
-    base = ["-std=c11", "-O2", "-fPIC", "-shared", "-Wall", "-o", LIB + ".tmp", SRC, "-lm"]
+    base = ["-std=c11", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-Wall", "-o", LIB + ".tmp", SRC, "-lm"]
     tried = []
     for cc in ("/usr/bin/gcc", "gcc", os.environ.get("CC", "cc")):
         for omp in (["-fopenmp"], []):

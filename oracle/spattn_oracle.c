@@ -64,11 +64,12 @@ typedef struct {
 typedef struct {
     int sink_blocks;    /* S */
     int local_blocks;   /* W */
-    int mode;           /* 0: top-k, 1: top-p */
+    int mode;           /* 0: top-k, 1: top-p, 2: top-p with the anchor-adaptive cap */
     int top_k;          /* top-k: fixed k when > 0 */
     double top_p;       /* top-p: mass threshold in (0, 1] */
     double max_ratio;   /* cap k_max = floor(max_ratio * n_mid); <= 0: no cap */
     double sm_scale;    /* 0: 1/sqrt(d) */
+    double min_ratio;   /* mode 2: the cap ratio when the anchors dominate */
 } spo_params;
 
 /* ---------------------------------------------------------------- decoding */
@@ -185,7 +186,9 @@ int spo_block_scores(const spo_dims *dm, const spo_params *pr, const uint16_t *q
         for (int c = 0; c < D; ++c)
             qbar[c] /= (double)G;
         for (int j = 0; j < dm->max_blocks; ++j) {
-            if (j < pr->sink_blocks || j >= nb - pr->local_blocks) {
+            /* mode 2 also scores the anchors (sink and local blocks) */
+            const int anchor = j < pr->sink_blocks || j >= nb - pr->local_blocks;
+            if (j >= nb || (anchor && pr->mode != 2)) {
                 out[j] = -INFINITY;
                 continue;
             }
@@ -216,8 +219,45 @@ static int rank_cmp(const void *a, const void *b)
     return (x->j > y->j) - (x->j < y->j);
 }
 
-/* Number of middle blocks kept for one query row, and the decision margin. */
-static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid,
+/*
+ * Mode 2 cap ("Claude Opus 长上下文 KV Cache 稀疏注意力", §多上下文场景下的跨文档注意力
+ * 恢复: the sink and local blocks are anchors; the maximum and minimum of the
+ * scores set the Top-P ratio, higher when the maximum stands well above the
+ * anchors).  Reading: a = the anchors' best score, hi / lo the middle's best
+ * and worst; r = clamp((hi - a) / (hi - lo), 0, 1) (0 when hi <= lo);
+ * ratio = min_ratio + r (max_ratio - min_ratio); k_max = floor(ratio n_mid).
+ * *margin_k: how far (in score units) the inputs may move before k_max
+ * changes.
+ */
+static int anchor_k_max(const spo_params *pr, double a, double hi, double lo, int n_mid, double *margin_k)
+{
+    double r = hi > lo ? (hi - a) / (hi - lo) : 0.0;
+    if (r < 0.0) r = 0.0;
+    if (r > 1.0) r = 1.0;
+    const double span = pr->max_ratio - pr->min_ratio;
+    const double ratio = pr->min_ratio + r * span;
+    const double x = ratio * (double)n_mid;
+    int k = (int)floor(x);
+    if (k > n_mid) k = n_mid;
+    if (!(hi > lo))
+        *margin_k = 0.0;                       /* degenerate: any change moves r */
+    else if (a >= hi)
+        *margin_k = a - hi;                    /* r pinned at 0 */
+    else if (a <= lo)
+        *margin_k = lo - a;                    /* r pinned at 1 */
+    else if (span <= 0.0)
+        *margin_k = INFINITY;
+    else {
+        double d = x - floor(x);
+        if (ceil(x) - x < d) d = ceil(x) - x;
+        *margin_k = d * (hi - lo) / (span * (double)n_mid);
+    }
+    return k;
+}
+
+/* Number of middle blocks kept for one query row, and the decision margin.
+ * a: the anchors' best score (mode 2 only). */
+static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid, double a,
                           double *margin)
 {
     int k_max = pr->max_ratio > 0.0 ? (int)floor(pr->max_ratio * (double)n_mid) : n_mid;
@@ -226,6 +266,9 @@ static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid,
     *margin = gap_inf;
     if (n_mid == 0)
         return 0;
+    double margin_k = INFINITY;
+    if (pr->mode == 2)
+        k_max = anchor_k_max(pr, a, r[0].s, r[n_mid - 1].s, n_mid, &margin_k);
     if (pr->mode == 0) {
         /* top-k: k = top_k if given, else the ratio's k_max; never above the
          * cap or the middle count. */
@@ -260,7 +303,7 @@ static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid,
         double mg = pr->top_p - cum;
         if (k_max > 0 && k_max < n_mid && r[k_max - 1].s - r[k_max].s < mg)
             mg = r[k_max - 1].s - r[k_max].s;
-        *margin = mg;
+        *margin = mg < margin_k ? mg : margin_k;
         return k_max;
     }
     double mg = pr->top_p - c_prev;
@@ -268,6 +311,9 @@ static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid,
         mg = c - pr->top_p;
     if (m < n_mid && r[m - 1].s - r[m].s < mg)
         mg = r[m - 1].s - r[m].s;
+    /* (k_max only matters when it binds, but a moved k_max could bind) */
+    if (pr->mode == 2 && m >= k_max - 1 && margin_k < mg)
+        mg = margin_k;
     *margin = mg;
     return m;
 }
@@ -304,8 +350,12 @@ int spo_select(const spo_dims *dm, const spo_params *pr, const double *scores,
                 r[i].j = S + i;
             }
             qsort(r, (size_t)n_mid, sizeof(ranked), rank_cmp);
+            double a = -INFINITY;   /* the anchors' best score (mode 2) */
+            if (pr->mode == 2)
+                for (int j = 0; j < nb; ++j)
+                    if ((j < S || j >= nb - W) && s[j] > a) a = s[j];
             double mg;
-            int m = row_keep_count(pr, r, n_mid, &mg);
+            int m = row_keep_count(pr, r, n_mid, a, &mg);
             if (mg < mg_row) mg_row = mg;
             for (int i = 0; i < m; ++i)
                 keep[r[i].j] = 1;

@@ -25,6 +25,13 @@ CHUNK2_TOPP = Workload("chunk2_topp", batch=2, q_tokens=2, num_q_heads=8, num_kv
                        seq_len=64 * 50 + 63, structure="zipf", mode="topp", top_p=0.9,
                        max_ratio=0.15, seed=17)
 GQA4_128K_SMALL = WORKLOADS["decode_128k_b2"]
+# anchor-adaptive cap (ratio 10-20 % of the middle blocks)
+SMALL_ANCHOR = Workload("small_anchor", batch=3, q_tokens=1, num_q_heads=8, num_kv_heads=2,
+                        seq_len=64 * 120 + 9, structure="zipf", mode="topp_anchor", top_p=0.9,
+                        min_ratio=0.10, max_ratio=0.20, seed=18)
+CHUNK2_ANCHOR = Workload("chunk2_anchor", batch=2, q_tokens=2, num_q_heads=16, num_kv_heads=4,
+                         seq_len=64 * 90 + 40, structure="planted", n_planted=8, mode="topp_anchor",
+                         top_p=0.8, min_ratio=0.05, max_ratio=0.25, seed=19)
 
 SMALL_CASES = [WORKLOADS["tiny_4k_gqa4"], SMALL_TOPP, SMALL_FP8_CHUNK, SMALL_RAGGED, GQA8_TOPP,
-               MQA16_TOPK, CHUNK16_FP8, CHUNK2_TOPP, GQA4_128K_SMALL]
+               MQA16_TOPK, CHUNK16_FP8, CHUNK2_TOPP, GQA4_128K_SMALL, SMALL_ANCHOR, CHUNK2_ANCHOR]

@@ -29,8 +29,12 @@ def dims_of(inp: dict, max_sel: int | None = None) -> oracle.Dims:
 
 
 def params_of(w, **kw) -> oracle.Params:
+    """The oracle's parameters as the library receives them: the fp32 values
+    of the float fields (so a ratio gives the same floor on both sides)."""
+    f32 = lambda x: float(np.float32(x))
     p = oracle.Params(sink_blocks=w.sink_blocks, local_blocks=w.local_blocks, mode=w.mode,
-                      top_k=w.top_k, top_p=w.top_p, max_ratio=w.max_ratio)
+                      top_k=w.top_k, top_p=f32(w.top_p), max_ratio=f32(w.max_ratio),
+                      min_ratio=f32(w.min_ratio))
     for k, v in kw.items():
         setattr(p, k, v)
     return p

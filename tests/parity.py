@@ -28,7 +28,7 @@ OUT_TOL = {False: 2e-3, True: 2e-2}
 
 def lib_params(w) -> spattn.Params:
     return spattn.Params(sink_blocks=w.sink_blocks, local_blocks=w.local_blocks, mode=w.mode,
-                         top_k=w.top_k, top_p=w.top_p, max_ratio=w.max_ratio)
+                         top_k=w.top_k, top_p=w.top_p, max_ratio=w.max_ratio, min_ratio=w.min_ratio)
 
 
 def run_library(inp: dict, params: spattn.Params | None = None) -> dict:
@@ -80,6 +80,19 @@ def subproblem(inp: dict, b: int) -> dict:
     return sub
 
 
+def anchor_cap(w, row_scores: np.ndarray, S: int, nb: int) -> int:
+    """The anchor-adaptive cap of one score row, computed as the library does
+    (double arithmetic on the fp32 scores and parameters)."""
+    W = w.local_blocks
+    mid = row_scores[S:nb - W].astype(np.float64)
+    a = max([float(row_scores[j]) for j in list(range(S)) + list(range(nb - W, nb))], default=-math.inf)
+    hi, lo = float(mid.max()), float(mid.min())
+    r = (hi - a) / (hi - lo) if hi > lo else 0.0
+    r = min(max(r, 0.0), 1.0)
+    mn, mx = float(np.float32(w.min_ratio)), float(np.float32(w.max_ratio))
+    return min(len(mid), math.floor((mn + r * (mx - mn)) * len(mid)))
+
+
 def _topp_prefix_ok(w, row_scores: np.ndarray, S: int, nb: int, got_mid: list[int]) -> bool:
     """GPU top-p set is the ranked prefix of its own scores of a length that
     sits within the fp32 rounding band of p (or at the cap)."""
@@ -91,7 +104,10 @@ def _topp_prefix_ok(w, row_scores: np.ndarray, S: int, nb: int, got_mid: list[in
         return False
     e = np.exp(s[order] - s[order[0]])
     c = np.cumsum(e / e.sum())
-    k_max = math.floor(w.max_ratio * len(mid)) if w.max_ratio > 0 else len(mid)
+    if w.mode == "topp_anchor":
+        k_max = anchor_cap(w, row_scores, S, nb)
+    else:
+        k_max = math.floor(w.max_ratio * len(mid)) if w.max_ratio > 0 else len(mid)
     if m == k_max:
         return True
     near = [abs(c[i] - w.top_p) for i in (m - 2, m - 1) if 0 <= i < len(c)]
@@ -154,7 +170,7 @@ def compare(inp: dict, gpu: dict, requests=None, params_override=None) -> dict:
             else:
                 want = sel_r[0, h, :cnt_r[0, h]].tolist()
                 if got != want:
-                    assert w.mode == "topp" and w.q_tokens == 1, f"replay b={b} h={h} differs"
+                    assert w.mode in ("topp", "topp_anchor") and w.q_tokens == 1, f"replay b={b} h={h} differs"
                     keep = set(range(min(w.sink_blocks, nb))) | set(range(max(0, nb - w.local_blocks), nb))
                     got_mid = [j for j in got if j not in keep]
                     assert _topp_prefix_ok(w, sc_g[0, 0, h], w.sink_blocks, nb, got_mid), \

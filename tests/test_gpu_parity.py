@@ -36,6 +36,7 @@ FULL = {
     "ragged_b32": None,          # shortest and longest request, chosen below
     "decode_1m_mqa": [1],
     "chunk16_fp8_512k": [2],
+    "decode_128k_b8_anchor": [3],
 }
 
 
