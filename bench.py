@@ -145,7 +145,9 @@ def step_bytes(inp, sel_count: torch.Tensor) -> dict:
     kv = kept * P * D * elt * 2 + (kept * 8 if w.kv_fp8 else 0)
     n_mid = sum(max(0, (int(L) + P - 1) // P - w.sink_blocks - w.local_blocks)
                 for L in inp["seq_lens"].tolist())
-    kbar = n_mid * H * D * 4
+    if w.mode == "topp_anchor":     # the anchor blocks are scored too
+        n_mid += sum(min((int(L) + P - 1) // P, w.sink_blocks + w.local_blocks) for L in inp["seq_lens"].tolist())
+    kbar = n_mid * H * D * (2 if w.kbar_bf16 else 4)
     q = inp["q"].numel() * 2
     out = inp["q"].numel() * 4
     return dict(kv=kv, kbar=kbar, q=q, out=out, total=kv + kbar + q + out, kept_block_heads=kept)
@@ -183,7 +185,8 @@ def run_native(args, rank, world, local_rank):
     max_sel = spattn.required_max_sel(dims, params)
     dims.max_sel = max_sel
     B, Tq, Hkv = w.batch, w.q_tokens, w.num_kv_heads
-    kbar = torch.empty((kc.shape[0], Hkv, w.head_dim), dtype=torch.float32, device=dev)
+    kbar = torch.empty((kc.shape[0], Hkv, w.head_dim), dtype=torch.bfloat16 if w.kbar_bf16 else torch.float32,
+                       device=dev)
     spattn.compress_keys(kc, ks, bt, sl, kbar, num_q_heads=w.num_q_heads, q_tokens=Tq)
     old_lens = (sl - Tq).clamp_min(0).to(torch.int32)
     scores = torch.empty((B, Tq, Hkv, bt.shape[1]), dtype=torch.float32, device=dev)
@@ -340,9 +343,39 @@ def run_native(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "wall_s": round(t_wall, 3),
     }
+    if w.kbar_bf16:
+        line["recall_vs_fp32_kbar"] = kbar_recall(inp, params, sel_idx, sel_count, dev)
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(inp, bts, ms_per_step)
     return line
+
+
+def kbar_recall(inp, params, sel_idx, sel_count, dev) -> float:
+    """Low-precision scoring, measured (outside the timed region): the share
+    of the middle blocks selected from fp32 compressed keys that the bf16
+    keys' selection also keeps, over every (request, KV head)."""
+    from block_sparse_kv_spattn_b200 import spattn
+    w = inp["workload"]
+    q, kc, bt, sl = inp["q"], inp["k_cache"], inp["block_table"], inp["seq_lens"]
+    kb32 = torch.empty((kc.shape[0], w.num_kv_heads, w.head_dim), dtype=torch.float32, device=dev)
+    spattn.compress_keys(kc, inp["k_scale"], bt, sl, kb32, num_q_heads=w.num_q_heads, q_tokens=w.q_tokens)
+    sc = torch.empty((w.batch, w.q_tokens, w.num_kv_heads, bt.shape[1]), dtype=torch.float32, device=dev)
+    si = torch.empty_like(sel_idx)
+    cnt = torch.empty_like(sel_count)
+    spattn.block_scores(q, kb32, bt, sl, sc, params, k_cache=kc)
+    spattn.select(sc, sl, si, cnt, params, q=q, k_cache=kc, block_table=bt)
+    torch.cuda.synchronize()
+    P = w.block_size
+    hit = total = 0
+    for b in range(w.batch):
+        nb = (int(sl[b]) + P - 1) // P
+        anchors = set(range(w.sink_blocks)) | set(range(nb - w.local_blocks, nb))
+        for h in range(w.num_kv_heads):
+            ref = set(si[b, h, :int(cnt[b, h])].tolist()) - anchors
+            got = set(sel_idx[b, h, :int(sel_count[b, h])].tolist()) - anchors
+            hit += len(ref & got)
+            total += len(ref)
+    return round(hit / max(1, total), 5)
 
 
 def cpu_baseline(inp, bts, gpu_ms):

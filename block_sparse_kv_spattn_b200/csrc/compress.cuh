@@ -16,8 +16,8 @@ struct CompressArgs {
     const int32_t *block_table;
     const int32_t *old_lens;  // nullable
     const int32_t *seq_lens;
-    float *kbar;              // [num_pages][Hkv][D]
-    int hkv, num_pages, max_blocks;
+    void *kbar;               // [num_pages][Hkv][D] fp32, or bf16 when kbar_bf16
+    int hkv, num_pages, max_blocks, kbar_bf16;
 };
 
 // Token groups per CTA so that a CTA has up to 512 threads.
@@ -91,9 +91,23 @@ __global__ void __launch_bounds__(512) compress_keys_kernel(CompressArgs a) {
             }
             const float sc = FP8 ? a.k_scale[(int64_t)page * a.hkv + h] : 1.f;
             const float n = (float)filled;
-            float4 *dst = reinterpret_cast<float4 *>(a.kbar + ((int64_t)page * a.hkv + h) * kHeadDim + chunk * 8);
-            dst[0] = make_float4(x.x * sc / n, x.y * sc / n, x.z * sc / n, x.w * sc / n);
-            dst[1] = make_float4(y.x * sc / n, y.y * sc / n, y.z * sc / n, y.w * sc / n);
+            const int64_t at = ((int64_t)page * a.hkv + h) * kHeadDim + chunk * 8;
+            const float m[8] = {x.x * sc / n, x.y * sc / n, x.z * sc / n, x.w * sc / n,
+                                y.x * sc / n, y.y * sc / n, y.z * sc / n, y.w * sc / n};
+            if (a.kbar_bf16) {
+                // the fp32 mean rounded to bf16 (nearest even)
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 v = __floats2bfloat162_rn(m[2 * e], m[2 * e + 1]);
+                    w[e] = *reinterpret_cast<const uint32_t *>(&v);
+                }
+                *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.kbar) + at) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.kbar) + at);
+                dst[0] = make_float4(m[0], m[1], m[2], m[3]);
+                dst[1] = make_float4(m[4], m[5], m[6], m[7]);
+            }
         }
         __syncthreads();
     }

@@ -14,7 +14,7 @@ namespace spattn {
 
 struct ScoresArgs {
     const uint16_t *q;        // bf16 bits [B][Tq][Hq][D]
-    const float *kbar;        // [num_pages][Hkv][D]
+    const void *kbar;         // [num_pages][Hkv][D] fp32, or bf16 (KB16)
     const int32_t *block_table;
     const int32_t *seq_lens;
     float *scores;            // [B][Tq][Hkv][max_blocks]
@@ -59,7 +59,7 @@ __device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
 // alongside the query rows.
 // Warp w takes blocks w, w + 4, ... of the CTA's range, BIF of them at a
 // time with all their compressed-key loads issued together.
-template <int HKV>
+template <int HKV, bool KB16>
 __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs a) {
     constexpr int BIF = HKV >= 16 ? 1 : (HKV >= 8 ? 2 : 4);
     constexpr int NW = kScoreThreads / 32;
@@ -131,9 +131,22 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
             const int page = jj < a.bpc ? pages[jj] : -1;
             mid[f] = page >= 0;
             if (mid[f]) {
-                const float4 *kp = reinterpret_cast<const float4 *>(a.kbar + (int64_t)page * HKV * kHeadDim);
+                if (KB16) {
+                    // 4 bf16 per lane: exact widening to fp32
+                    const uint2 *kp = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.kbar) +
+                                                                      (int64_t)page * HKV * kHeadDim);
 #pragma unroll
-                for (int hh = 0; hh < HKV; ++hh) kv[f][hh] = kp[hh * (kHeadDim / 4) + lane];
+                    for (int hh = 0; hh < HKV; ++hh) {
+                        const uint2 u = kp[hh * (kHeadDim / 4) + lane];
+                        kv[f][hh] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+                    }
+                } else {
+                    const float4 *kp = reinterpret_cast<const float4 *>(static_cast<const float *>(a.kbar) +
+                                                                        (int64_t)page * HKV * kHeadDim);
+#pragma unroll
+                    for (int hh = 0; hh < HKV; ++hh) kv[f][hh] = kp[hh * (kHeadDim / 4) + lane];
+                }
             }
         }
 #pragma unroll

@@ -77,6 +77,8 @@ spattn_status check_dims(const spattn_dims *d) {
                     d->num_q_heads, d->num_kv_heads);
     if (!pow2_hkv(d->num_kv_heads))
         return fail(SPATTN_ERR_UNSUPPORTED, "num_kv_heads %d: built for 1, 2, 4, 8, 16", d->num_kv_heads);
+    if (d->kbar_dtype != SPATTN_KBAR_F32 && d->kbar_dtype != SPATTN_KBAR_BF16)
+        return fail(SPATTN_ERR_INVALID_ARG, "kbar_dtype %d", d->kbar_dtype);
     const int64_t rows = (int64_t)d->q_tokens * (d->num_q_heads / d->num_kv_heads);
     if (rows > 64)
         return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_q_heads / num_kv_heads = %lld > 64",
@@ -231,7 +233,7 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 }
 
 spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const void *q,
-                            const float *kbar, const int32_t *bt, const int32_t *sl, float *scores,
+                            const void *kbar, const int32_t *bt, const int32_t *sl, float *scores,
                             cudaStream_t st) {
     ScoresArgs a;
     a.q = static_cast<const uint16_t *>(q);
@@ -253,23 +255,30 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     if (smem > kMaxSmem)
         return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_kv_heads = %d too large for block scores", rowsq);
     dim3 grid((d->max_blocks_per_seq + a.bpc - 1) / a.bpc, d->batch);
+    const bool kb16 = d->kbar_dtype == SPATTN_KBAR_BF16;
     const void *fn = nullptr;
+#define SP_SCORES_FN(H) (kb16 ? (const void *)block_scores_kernel<H, true> : (const void *)block_scores_kernel<H, false>)
     switch (d->num_kv_heads) {
-        case 1: fn = (const void *)block_scores_kernel<1>; break;
-        case 2: fn = (const void *)block_scores_kernel<2>; break;
-        case 4: fn = (const void *)block_scores_kernel<4>; break;
-        case 8: fn = (const void *)block_scores_kernel<8>; break;
-        case 16: fn = (const void *)block_scores_kernel<16>; break;
+        case 1: fn = SP_SCORES_FN(1); break;
+        case 2: fn = SP_SCORES_FN(2); break;
+        case 4: fn = SP_SCORES_FN(4); break;
+        case 8: fn = SP_SCORES_FN(8); break;
+        case 16: fn = SP_SCORES_FN(16); break;
     }
+#undef SP_SCORES_FN
     SP_TRY(ensure_smem(fn, smem));
     cudaError_t e = cudaSuccess;
+#define SP_SCORES_LAUNCH(H)                                                                     \
+    e = kb16 ? launch(block_scores_kernel<H, true>, grid, kScoreThreads, smem, st, a)          \
+             : launch(block_scores_kernel<H, false>, grid, kScoreThreads, smem, st, a)
     switch (d->num_kv_heads) {
-        case 1: e = launch(block_scores_kernel<1>, grid, kScoreThreads, smem, st, a); break;
-        case 2: e = launch(block_scores_kernel<2>, grid, kScoreThreads, smem, st, a); break;
-        case 4: e = launch(block_scores_kernel<4>, grid, kScoreThreads, smem, st, a); break;
-        case 8: e = launch(block_scores_kernel<8>, grid, kScoreThreads, smem, st, a); break;
-        case 16: e = launch(block_scores_kernel<16>, grid, kScoreThreads, smem, st, a); break;
+        case 1: SP_SCORES_LAUNCH(1); break;
+        case 2: SP_SCORES_LAUNCH(2); break;
+        case 4: SP_SCORES_LAUNCH(4); break;
+        case 8: SP_SCORES_LAUNCH(8); break;
+        case 16: SP_SCORES_LAUNCH(16); break;
     }
+#undef SP_SCORES_LAUNCH
     return cuda_ok(e, "block_scores launch");
 }
 
@@ -544,7 +553,7 @@ int32_t spattn_required_max_sel(const spattn_dims *dims, const spattn_params *pa
 
 spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache, const float *k_scale,
                                    const int32_t *block_table, const int32_t *old_lens,
-                                   const int32_t *seq_lens, float *kbar, spattn_stream_t stream) {
+                                   const int32_t *seq_lens, void *kbar, spattn_stream_t stream) {
     SP_TRY(check_dims(dims));
     if (!k_cache || !block_table || !seq_lens || !kbar)
         return fail(SPATTN_ERR_INVALID_ARG, "k_cache, block_table, seq_lens, kbar are required");
@@ -559,6 +568,7 @@ spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache,
     a.old_lens = old_lens;
     a.seq_lens = seq_lens;
     a.kbar = kbar;
+    a.kbar_bf16 = dims->kbar_dtype == SPATTN_KBAR_BF16;
     a.hkv = dims->num_kv_heads;
     a.num_pages = dims->num_pages;
     a.max_blocks = dims->max_blocks_per_seq;
@@ -580,7 +590,7 @@ spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache,
 }
 
 spattn_status spattn_block_scores(const spattn_dims *dims, const spattn_params *params, const void *q,
-                                  const float *kbar, const int32_t *block_table,
+                                  const void *kbar, const int32_t *block_table,
                                   const int32_t *seq_lens, float *scores, spattn_stream_t stream) {
     SP_TRY(check_dims(dims));
     SP_TRY(check_params(params));
@@ -664,7 +674,7 @@ spattn_status spattn_decode_selected_noalloc(const spattn_dims *dims, const spat
 spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params, const void *q,
                             const void *k_cache, const void *v_cache, const float *k_scale,
                             const float *v_scale, const int32_t *block_table, const int32_t *seq_lens,
-                            const float *kbar, float *out, int32_t *sel_idx, int32_t *sel_count,
+                            const void *kbar, float *out, int32_t *sel_idx, int32_t *sel_count,
                             float *scores_out, void *workspace, size_t workspace_bytes,
                             spattn_stream_t stream) {
     SP_TRY(check_dims(dims));

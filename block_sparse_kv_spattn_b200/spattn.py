@@ -31,6 +31,7 @@ DEV_BAD_PAGE, DEV_BAD_BLOCK, DEV_SEL_OVERFLOW, DEV_WAIT_TIMEOUT, DEV_BAD_LEN = 1
 KV_BF16, KV_FP8_E4M3 = 0, 1
 SEL_TOPK, SEL_TOPP, SEL_TOPP_ANCHOR = 0, 1, 2
 SEL_MODES = {"topk": SEL_TOPK, "topp": SEL_TOPP, "topp_anchor": SEL_TOPP_ANCHOR}
+KBAR_F32, KBAR_BF16 = 0, 1
 
 EXPORTS = ("spattn_required_max_sel", "spattn_compress_keys", "spattn_block_scores",
            "spattn_select", "spattn_decode_workspace_size", "spattn_decode_selected",
@@ -47,7 +48,7 @@ class SpattnError(RuntimeError):
 class CDims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "q_tokens", "num_q_heads", "num_kv_heads", "head_dim", "block_size",
-        "num_pages", "max_blocks_per_seq", "max_sel", "kv_dtype")]
+        "num_pages", "max_blocks_per_seq", "max_sel", "kv_dtype", "kbar_dtype")]
 
 
 class CParams(ctypes.Structure):
@@ -128,12 +129,17 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def kbar_dtype_of(kbar) -> int:
+    """fp32 compressed keys, or bf16 (low-precision scoring)."""
+    return KBAR_BF16 if kbar is not None and kbar.dtype == torch.bfloat16 else KBAR_F32
+
+
 def dims_for(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor,
-             max_sel: int = 0) -> CDims:
+             max_sel: int = 0, kbar=None) -> CDims:
     B, Tq, Hq, D = q.shape
     num_pages, Hkv, P, D2 = k_cache.shape
     kv = KV_FP8_E4M3 if k_cache.dtype in (torch.uint8, torch.float8_e4m3fn) else KV_BF16
-    return CDims(B, Tq, Hq, Hkv, D, P, num_pages, block_table.shape[1], max_sel, kv)
+    return CDims(B, Tq, Hq, Hkv, D, P, num_pages, block_table.shape[1], max_sel, kv, kbar_dtype_of(kbar))
 
 
 def required_max_sel(dims: CDims, params: Params) -> int:
@@ -159,7 +165,7 @@ def compress_keys(k_cache, k_scale, block_table, seq_lens, kbar, old_lens=None, 
     num_pages, Hkv, P, D = k_cache.shape
     kv = KV_FP8_E4M3 if k_cache.dtype in (torch.uint8, torch.float8_e4m3fn) else KV_BF16
     dims = CDims(seq_lens.shape[0], q_tokens, max(num_q_heads, Hkv), Hkv, D, P, num_pages,
-                 block_table.shape[1], 0, kv)
+                 block_table.shape[1], 0, kv, kbar_dtype_of(kbar))
     _check(load().spattn_compress_keys(ctypes.byref(dims), _p(k_cache),
                                        _p(k_scale) if kv == KV_FP8_E4M3 else None,
                                        _p(block_table), _p(old_lens), _p(seq_lens), _p(kbar),
@@ -167,7 +173,7 @@ def compress_keys(k_cache, k_scale, block_table, seq_lens, kbar, old_lens=None, 
 
 
 def block_scores(q, kbar, block_table, seq_lens, scores, params: Params, *, k_cache, stream=None):
-    dims = dims_for(q, k_cache, block_table)
+    dims = dims_for(q, k_cache, block_table, kbar=kbar)
     _check(load().spattn_block_scores(ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(kbar),
                                       _p(block_table), _p(seq_lens), _p(scores), _stream(stream)))
 
@@ -204,7 +210,7 @@ def decode_selected_noalloc(q, k_cache, v_cache, k_scale, v_scale, block_table, 
 
 def decode(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, kbar, out, sel_idx,
            sel_count, workspace, params: Params, scores_out=None, stream=None):
-    dims = dims_for(q, k_cache, block_table, sel_idx.shape[-1])
+    dims = dims_for(q, k_cache, block_table, sel_idx.shape[-1], kbar=kbar)
     fp8 = dims.kv_dtype == KV_FP8_E4M3
     _check(load().spattn_decode(
         ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(k_cache), _p(v_cache),

@@ -54,6 +54,7 @@ class Workload:
     top_p: float = 1.0
     max_ratio: float = 0.0
     min_ratio: float = 0.0            # topp_anchor: the cap ratio when the anchors dominate
+    kbar_bf16: bool = False           # compressed keys stored as bf16 (low-precision scoring)
     sink_blocks: int = 1
     local_blocks: int = 2
     head_dim: int = HEAD_DIM
@@ -82,6 +83,10 @@ WORKLOADS = {
                                       num_kv_heads=8, seq_len=131072, structure="zipf",
                                       mode="topp_anchor", top_p=0.9, min_ratio=0.10, max_ratio=0.20,
                                       seed=1241),
+    # the gate shape scored from bf16 compressed keys (half the scoring bytes)
+    "decode_128k_b8_kbar16": Workload("decode_128k_b8_kbar16", batch=8, q_tokens=1, num_q_heads=32,
+                                      num_kv_heads=8, seq_len=131072, structure="zipf", mode="topp",
+                                      top_p=0.9, max_ratio=0.15, kbar_bf16=True, seed=1236),
     # the same shape with 2 requests: small enough for detailed profiling
     "decode_128k_b2": Workload("decode_128k_b2", batch=2, q_tokens=1, num_q_heads=32, num_kv_heads=8,
                                seq_len=131072, structure="zipf", mode="topp", top_p=0.9,

@@ -51,7 +51,8 @@
  *   block_table int32 [B][max_blocks_per_seq]  logical block j -> page id
  *   seq_lens   int32 [B]                   tokens in the cache, including
  *                                         the Tq query tokens
- *   kbar       f32   [num_pages][Hkv][d]   mean-pooled key of each page
+ *   kbar       f32 or bf16 (dims.kbar_dtype) [num_pages][Hkv][d]
+ *                                         mean-pooled key of each page
  *   scores     f32   [B][Tq][Hkv][max_blocks_per_seq]
  *   sel_idx    int32 [B][Hkv][max_sel]     kept logical block ids, ascending
  *   sel_count  int32 [B][Hkv]
@@ -90,6 +91,14 @@ typedef enum {
 
 typedef enum { SPATTN_KV_BF16 = 0, SPATTN_KV_FP8_E4M3 = 1 } spattn_kv_dtype;
 /*
+ * Storage of the compressed keys.  SPATTN_KBAR_BF16 halves the bytes the
+ * block scores read: the fp32 mean rounded to bf16 (nearest even), scores
+ * still accumulated in fp32 -- low-precision scoring after "CSA + HCA 混合注意力
+ * 机制" §4.2 (the indexer's QK path runs at low precision; the page reports
+ * 99.7 % top-k recall against BF16 for its FP4 path).
+ */
+typedef enum { SPATTN_KBAR_F32 = 0, SPATTN_KBAR_BF16 = 1 } spattn_kbar_dtype;
+/*
  * Selection modes.  SPATTN_SEL_TOPP_ANCHOR: top-p whose retention cap adapts
  * to the anchors ("Claude Opus 长上下文 KV Cache 稀疏注意力", §多上下文场景下的跨文档
  * 注意力恢复, anchor-based dynamic selection: the sink and local blocks are
@@ -116,6 +125,7 @@ typedef struct {
     int32_t max_blocks_per_seq; /* columns of block_table and scores */
     int32_t max_sel;            /* columns of sel_idx; >= spattn_required_max_sel() */
     int32_t kv_dtype;           /* spattn_kv_dtype */
+    int32_t kbar_dtype;         /* spattn_kbar_dtype of kbar */
 } spattn_dims;
 
 typedef struct {
@@ -163,7 +173,7 @@ int32_t spattn_required_max_sel(const spattn_dims *dims, const spattn_params *pa
 spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache,
                                    const float *k_scale, const int32_t *block_table,
                                    const int32_t *old_lens, const int32_t *seq_lens,
-                                   float *kbar, spattn_stream_t stream);
+                                   void *kbar, spattn_stream_t stream);
 
 /*
  * spattn_block_scores -- score every middle block.
@@ -175,7 +185,7 @@ spattn_status spattn_compress_keys(const spattn_dims *dims, const void *k_cache,
  * past the end).  fp32 arithmetic throughout.
  */
 spattn_status spattn_block_scores(const spattn_dims *dims, const spattn_params *params,
-                                  const void *q, const float *kbar,
+                                  const void *q, const void *kbar,
                                   const int32_t *block_table, const int32_t *seq_lens,
                                   float *scores, spattn_stream_t stream);
 
@@ -264,7 +274,7 @@ spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params
                             const void *q, const void *k_cache, const void *v_cache,
                             const float *k_scale, const float *v_scale,
                             const int32_t *block_table, const int32_t *seq_lens,
-                            const float *kbar, float *out, int32_t *sel_idx,
+                            const void *kbar, float *out, int32_t *sel_idx,
                             int32_t *sel_count, float *scores_out, void *workspace,
                             size_t workspace_bytes, spattn_stream_t stream);
 

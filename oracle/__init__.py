@@ -92,6 +92,10 @@ def lib():
         L.spo_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         L.spo_e4m3_to_f64.restype = ctypes.c_double
         L.spo_num_threads.restype = ctypes.c_int
+        L.spo_round_bf16.argtypes = [ctypes.c_double]
+        L.spo_round_bf16.restype = ctypes.c_double
+        L.spo_round_bf16_array.argtypes = [P, ctypes.c_int64]
+        L.spo_round_bf16_array.restype = None
         _lib = L
     return _lib
 
@@ -114,6 +118,16 @@ def bf16_to_f64(bits: int) -> float:
 
 def e4m3_to_f64(bits: int) -> float:
     return lib().spo_e4m3_to_f64(bits)
+
+
+def round_bf16(x):
+    """The nearest bf16 values (ties to even) of float64 data, as float64:
+    the compressed keys of low-precision scoring."""
+    if np.isscalar(x):
+        return lib().spo_round_bf16(float(x))
+    a = np.array(x, dtype=np.float64, copy=True, order="C")
+    lib().spo_round_bf16_array(_ptr(a), a.size)
+    return a
 
 
 def _cache_dtype(dims: Dims):

@@ -74,6 +74,33 @@ typedef struct {
 
 /* ---------------------------------------------------------------- decoding */
 
+/*
+ * The bf16 value nearest to x, ties to even: bf16 keeps the top 16 bits of a
+ * binary32, i.e. 8 significant bits with binary32's exponent range (smallest
+ * normal 2^-126, subnormal spacing 2^-133, largest finite (2 - 2^-7) 2^127).
+ * One rounding from binary64 (low-precision scoring: "CSA + HCA 混合注意力机制"
+ * §4.2, the indexer's QK path at reduced precision).
+ */
+double spo_round_bf16(double x)
+{
+    if (!isfinite(x) || x == 0.0)
+        return x;
+    int e;
+    (void)frexp(x, &e);                 /* |x| = m 2^e, m in [0.5, 1) */
+    int q = e - 8;                      /* spacing of 8-bit significands in this binade */
+    if (q < -133) q = -133;             /* subnormal: fixed spacing */
+    double y = ldexp(nearbyint(ldexp(x, -q)), q);   /* exact scalings; nearbyint ties to even */
+    if (fabs(y) >= 0x1p128)
+        y = copysign(INFINITY, x);
+    return y;
+}
+
+void spo_round_bf16_array(double *x, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        x[i] = spo_round_bf16(x[i]);
+}
+
 /* bf16 is the high 16 bits of a binary32: widening is exact. */
 double spo_bf16_to_f64(uint16_t bits)
 {

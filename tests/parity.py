@@ -1,7 +1,10 @@
 """Run the CUDA library and the float64 oracle on the same bytes and compare.
 
 Tolerances (derived in the design notes from fp32 arithmetic):
-  kbar    |gpu - oracle| <= 2e-6 * max|column| + 1e-7 * |oracle|
+  kbar    |gpu - oracle| <= 2e-6 * max|column| + 1e-7 * |oracle|; bf16 compressed
+          keys: the oracle's mean rounded to bf16, within one bf16 step
+          (2^-7 |oracle|) on top of that, and the scores checked against the
+          oracle's scoring of the GPU's own compressed keys
   scores  |gpu - oracle| <= 1e-5 * max(1, |oracle|)
   indices bit-exact where the oracle's decision margin exceeds 1e-4;
           otherwise replayed: the oracle's selection run on the GPU's own
@@ -31,14 +34,15 @@ def lib_params(w) -> spattn.Params:
                          top_k=w.top_k, top_p=w.top_p, max_ratio=w.max_ratio, min_ratio=w.min_ratio)
 
 
-def run_library(inp: dict, params: spattn.Params | None = None) -> dict:
+def run_library(inp: dict, params: spattn.Params | None = None, kbar_bf16: bool = False) -> dict:
     """compress (all blocks) + decode through the C ABI; results on device."""
     w = inp["workload"]
     params = params or lib_params(w)
     q, kc, vc = inp["q"], inp["k_cache"], inp["v_cache"]
     bt, sl = inp["block_table"], inp["seq_lens"]
     dev = q.device
-    kbar = torch.full((kc.shape[0], kc.shape[1], kc.shape[3]), float("nan"), device=dev)
+    kbar = torch.full((kc.shape[0], kc.shape[1], kc.shape[3]), float("nan"), device=dev,
+                      dtype=torch.bfloat16 if kbar_bf16 else torch.float32)
     spattn.compress_keys(kc, inp["k_scale"], bt, sl, kbar, num_q_heads=w.num_q_heads,
                          q_tokens=w.q_tokens)
     dims = spattn.dims_for(q, kc, bt)
@@ -114,7 +118,7 @@ def _topp_prefix_ok(w, row_scores: np.ndarray, S: int, nb: int, got_mid: list[in
     return bool(near) and min(near) < TOPP_BAND
 
 
-def compare(inp: dict, gpu: dict, requests=None, params_override=None) -> dict:
+def compare(inp: dict, gpu: dict, requests=None, params_override=None, kbar_bf16: bool = False) -> dict:
     """Compare every step for the listed requests (default: all).  Returns a
     summary (max errors, exact/replayed row counts); raises AssertionError on
     any violation."""
@@ -143,18 +147,24 @@ def compare(inp: dict, gpu: dict, requests=None, params_override=None) -> dict:
             filled = torch.clamp(L - torch.arange(nb, device=K.device) * P, max=P)
             tmask = (torch.arange(P, device=K.device)[None, :] < filled[:, None])[:, None, :, None]
             colmax = torch.where(tmask, K.abs(), torch.zeros_like(K)).amax(dim=2).cpu().numpy()
-            tol = 2e-6 * colmax + 1e-7 * np.abs(kb_o[:nb])
+            if kbar_bf16:
+                kb_o = oracle.round_bf16(kb_o)
+                tol = 2e-6 * colmax + 2.0 ** -7 * np.abs(kb_o[:nb]) + 1e-30
+            else:
+                tol = 2e-6 * colmax + 1e-7 * np.abs(kb_o[:nb])
             err = np.abs(kb_g - kb_o[:nb])
             assert np.all(err <= tol), f"kbar b={b}: max err {err.max():.3g}"
             summary["kbar_err"] = max(summary["kbar_err"], float(err.max()))
         # 2. scores
         sc_o = oracle.block_scores(dims, opar, qh, kb_o, bt, sl)
         sc_g = gpu["scores"][b:b + 1].double().cpu().numpy()
+        # the scoring itself: against the oracle's scores of the GPU's own keys
+        sc_c = oracle.block_scores(dims, opar, qh, kb_g, bt, sl) if kbar_bf16 and nb else sc_o
         fin = np.isfinite(sc_o)
         assert np.array_equal(fin, np.isfinite(sc_g)), f"scores b={b}: -inf pattern differs"
         if fin.any():
-            err = np.abs(sc_g[fin] - sc_o[fin])
-            assert np.all(err <= 1e-5 * np.maximum(1.0, np.abs(sc_o[fin]))), \
+            err = np.abs(sc_g[fin] - sc_c[fin])
+            assert np.all(err <= 1e-5 * np.maximum(1.0, np.abs(sc_c[fin]))), \
                 f"scores b={b}: max err {err.max():.3g}"
             summary["score_err"] = max(summary["score_err"], float(err.max()))
         # 3. selection: exact where the margin is clear, else replay

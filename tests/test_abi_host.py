@@ -39,7 +39,7 @@ def test_only_the_abi_is_exported():
 
 def _dims(**kw):
     d = dict(batch=2, q_tokens=1, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=64,
-             num_pages=100, max_blocks_per_seq=50, max_sel=50, kv_dtype=0)
+             num_pages=100, max_blocks_per_seq=50, max_sel=50, kv_dtype=0, kbar_dtype=0)
     d.update(kw)
     return spattn.CDims(*[d[n] for n, _ in spattn.CDims._fields_])
 

@@ -155,3 +155,39 @@ def test_decode_selected_with_given_selection():
                         cache_bytes(inp["v_cache"]), None, None, inp["block_table"].cpu().numpy(),
                         inp["seq_lens"].cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy())
     assert np.abs(out.double().cpu().numpy() - ref).max() <= 2e-3
+
+
+# ------------------------------------------ low-precision (bf16) compressed keys
+
+from tests.cases import GQA8_TOPP, MQA16_TOPK, SMALL_FP8_CHUNK, SMALL_TOPP  # noqa: E402
+
+
+@pytest.mark.parametrize("w", [SMALL_TOPP, GQA8_TOPP, MQA16_TOPK, SMALL_FP8_CHUNK], ids=lambda w: w.name)
+def test_bf16_kbar_parity(w):
+    """Compressed keys stored as bf16: keys within one bf16 step of the
+    oracle's rounded mean, scores equal to the oracle's scoring of those
+    keys, selection by the margin / replay rule, outputs within tolerance."""
+    inp = make_inputs(w, device="cuda")
+    gpu = run_library(inp, kbar_bf16=True)
+    assert gpu["kbar"].dtype == torch.bfloat16
+    s = compare(inp, gpu, kbar_bf16=True)
+    assert s["exact_rows"] + s["replayed_rows"] == w.batch * w.num_kv_heads
+
+
+def test_bf16_kbar_recall_at_128k():
+    """Low-precision scoring at full size: the share of the middle blocks the
+    fp32 keys select that the bf16 keys' selection keeps as well."""
+    w = WORKLOADS["decode_128k_b8"]
+    inp = make_inputs(w, device="cuda")
+    ref, low = run_library(inp), run_library(inp, kbar_bf16=True)
+    P, hit, total = w.block_size, 0, 0
+    for b in range(w.batch):
+        nb = (int(inp["seq_lens"][b]) + P - 1) // P
+        anchors = set(range(w.sink_blocks)) | set(range(nb - w.local_blocks, nb))
+        for h in range(w.num_kv_heads):
+            r = set(ref["sel_idx"][b, h, :int(ref["sel_count"][b, h])].tolist()) - anchors
+            g = set(low["sel_idx"][b, h, :int(low["sel_count"][b, h])].tolist()) - anchors
+            hit, total = hit + len(r & g), total + len(r)
+    recall = hit / total
+    print(f"bf16 compressed keys: middle-block recall {recall:.4f} over {total} blocks")
+    assert recall >= 0.9

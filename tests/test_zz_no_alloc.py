@@ -64,7 +64,7 @@ def test_noalloc_rejects_dims_beyond_its_scratch(cuda):
     """64 query rows per KV head over 128 requests x 8 KV heads need far more
     than the built-in scratch: refused on the host, nothing enqueued."""
     lib = spattn.load()
-    d = spattn.CDims(128, 16, 32, 8, 128, 64, 1000, 100, 100, 0)
+    d = spattn.CDims(128, 16, 32, 8, 128, 64, 1000, 100, 100, 0, 0)
     p = spattn.Params(top_k=4).c()
     dummy = ctypes.c_void_p(256)
     st = lib.spattn_decode_selected_noalloc(ctypes.byref(d), ctypes.byref(p), dummy, dummy, dummy,
