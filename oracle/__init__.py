@@ -82,7 +82,9 @@ def lib():
             "spo_compress_keys": [P, P, P, P, P, P],
             "spo_block_scores": [P, P, P, P, P, P, P],
             "spo_select": [P, P, P, P, P, P, P],
-            "spo_attend": [P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int, P],
+            "spo_attend": [P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int, P, P],
+            "spo_hca_pool": [P, P, P, P, P, P, P, ctypes.c_int, P, P],
+            "spo_hca_attend": [P, P, P, P, P, P, ctypes.c_int, P, P],
         }.items():
             fn = getattr(L, name)
             fn.argtypes = args
@@ -175,12 +177,14 @@ def select(dims: Dims, params: Params, scores, seq_lens):
 
 
 def attend(dims: Dims, params: Params, q, k_cache, v_cache, k_scale, v_scale,
-           block_table, seq_lens, sel_idx, sel_count, units=None) -> np.ndarray:
-    """Softmax attention over the kept blocks: float64 [B][Tq][Hq][d].
+           block_table, seq_lens, sel_idx, sel_count, units=None, with_lse=False):
+    """Softmax attention over the kept blocks: float64 [B][Tq][Hq][d]
+    (and, with_lse, the ln-sum-exp of each row's logits [B][Tq][Hq]).
 
     ``units``: optional list of (b, h) pairs to compute; other rows stay 0.
     """
     out = np.zeros((dims.batch, dims.q_tokens, dims.num_q_heads, dims.head_dim), np.float64)
+    lse = np.full((dims.batch, dims.q_tokens, dims.num_q_heads), -np.inf) if with_lse else None
     cd = _cache_dtype(dims)
     k_cache, v_cache = _c(k_cache, cd), _c(v_cache, cd)
     ks = _c(k_scale, np.float32) if dims.kv_fp8 else None
@@ -190,10 +194,52 @@ def attend(dims: Dims, params: Params, q, k_cache, v_cache, k_scale, v_scale,
                           _ptr(k_cache), _ptr(v_cache), _ptr(ks), _ptr(vs),
                           _ptr(_c(block_table, np.int32)), _ptr(_c(seq_lens, np.int32)),
                           _ptr(_c(sel_idx, np.int32)), _ptr(_c(sel_count, np.int32)),
-                          _ptr(u), 0 if u is None else len(u), _ptr(out))
+                          _ptr(u), 0 if u is None else len(u), _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError(f"spo_attend failed ({rc})")
-    return out
+    return (out, lse) if with_lse else out
+
+
+def hca_pool(dims: Dims, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, group_blocks=2):
+    """Mean-pooled K and V of every group of group_blocks logical blocks:
+    float64 [B][G_max][Hkv][d] each."""
+    gmax = (dims.max_blocks + group_blocks - 1) // group_blocks
+    khat = np.zeros((dims.batch, gmax, dims.num_kv_heads, dims.head_dim), np.float64)
+    vhat = np.zeros_like(khat)
+    cd = _cache_dtype(dims)
+    ks = _c(k_scale, np.float32) if dims.kv_fp8 else None
+    vs = _c(v_scale, np.float32) if dims.kv_fp8 else None
+    rc = lib().spo_hca_pool(ctypes.byref(dims.c()), _ptr(_c(k_cache, cd)), _ptr(_c(v_cache, cd)), _ptr(ks),
+                            _ptr(vs), _ptr(_c(block_table, np.int32)), _ptr(_c(seq_lens, np.int32)),
+                            group_blocks, _ptr(khat), _ptr(vhat))
+    if rc != 0:
+        raise ValueError(f"spo_hca_pool failed ({rc})")
+    return khat, vhat
+
+
+def hca_attend(dims: Dims, params: Params, q, khat, vhat, seq_lens, group_blocks=2):
+    """Dense attention over the pooled entries: (out [B][Tq][Hq][d], lse [B][Tq][Hq])."""
+    out = np.zeros((dims.batch, dims.q_tokens, dims.num_q_heads, dims.head_dim), np.float64)
+    lse = np.full((dims.batch, dims.q_tokens, dims.num_q_heads), -np.inf)
+    rc = lib().spo_hca_attend(ctypes.byref(dims.c()), ctypes.byref(params.c()), _ptr(_c(q, np.uint16)),
+                              _ptr(_c(khat, np.float64)), _ptr(_c(vhat, np.float64)),
+                              _ptr(_c(seq_lens, np.int32)), group_blocks, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"spo_hca_attend failed ({rc})")
+    return out, lse
+
+
+def lse_merge(out_a, lse_a, out_b, lse_b):
+    """Softmax over the union of two key sets from the two partial results:
+    out = (e^lse_a out_a + e^lse_b out_b) / (e^lse_a + e^lse_b), lse = ln of
+    the sum (a row with neither keeps 0 and -inf)."""
+    m = np.maximum(lse_a, lse_b)
+    mm = np.where(np.isfinite(m), m, 0.0)
+    wa, wb = np.exp(lse_a - mm), np.exp(lse_b - mm)
+    z = wa + wb
+    out = (wa[..., None] * out_a + wb[..., None] * out_b) / np.where(z > 0, z, 1.0)[..., None]
+    lse = np.where(z > 0, mm + np.log(np.where(z > 0, z, 1.0)), -np.inf)
+    return out, lse
 
 
 def decode(dims: Dims, params: Params, q, k_cache, v_cache, k_scale, v_scale,

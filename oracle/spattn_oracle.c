@@ -420,7 +420,7 @@ int spo_attend(const spo_dims *dm, const spo_params *pr, const uint16_t *q,
                const float *v_scale, const int32_t *block_table,
                const int32_t *seq_lens, const int32_t *sel_idx,
                const int32_t *sel_count, const int32_t *units, int n_units,
-               double *out)
+               double *out, double *lse)
 {
     const int D = dm->head_dim, H = dm->num_kv_heads, Tq = dm->q_tokens;
     const int P = dm->block_size, Hq = dm->num_q_heads, G = Hq / H;
@@ -463,6 +463,8 @@ int spo_attend(const spo_dims *dm, const spo_params *pr, const uint16_t *q,
                 }
                 for (int c = 0; c < D; ++c)
                     o[c] = 0.0;
+                double *ls = lse ? lse + (((int64_t)b * Tq + t) * Hq + i) : NULL;
+                if (ls) *ls = -INFINITY;
                 if (n == 0)
                     continue;
                 double mx = logit[0];
@@ -471,6 +473,7 @@ int spo_attend(const spo_dims *dm, const spo_params *pr, const uint16_t *q,
                 double z = 0.0;
                 for (int k = 0; k < n; ++k)
                     z += exp(logit[k] - mx);
+                if (ls) *ls = mx + log(z);   /* ln of the sum of exp(logit) */
                 for (int k = 0; k < n; ++k) {
                     double p = exp(logit[k] - mx) / z;
                     for (int c = 0; c < D; ++c)
@@ -481,6 +484,107 @@ int spo_attend(const spo_dims *dm, const spo_params *pr, const uint16_t *q,
         free(logit);
         free(tpage);
         free(tslot);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------- 6. HCA branch (weight-free) */
+
+/*
+ * "CSA + HCA 混合注意力机制" §5.1-5.2: every m' consecutive tokens are pooled
+ * into one entry and a query attends densely over all entries.  Reading: the
+ * pooling is the mean (the page's learned attention pooling needs weights);
+ * a group is group_blocks consecutive logical blocks (m' = group_blocks * P).
+ * khat/vhat[b][g][h][c] = mean over the group's filled tokens of K / V;
+ * groups past a request's end are 0.  Layout [B][G_max][H][D],
+ * G_max = ceil(max_blocks / group_blocks).
+ */
+int spo_hca_pool(const spo_dims *dm, const void *k_cache, const void *v_cache,
+                 const float *k_scale, const float *v_scale, const int32_t *block_table,
+                 const int32_t *seq_lens, int group_blocks, double *khat, double *vhat)
+{
+    const int D = dm->head_dim, H = dm->num_kv_heads, P = dm->block_size;
+    const int Gmax = (dm->max_blocks + group_blocks - 1) / group_blocks;
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t bg = 0; bg < (int64_t)dm->batch * Gmax; ++bg) {
+        int b = (int)(bg / Gmax), g = (int)(bg % Gmax);
+        int64_t L = seq_lens[b], t0 = (int64_t)g * group_blocks * P;
+        int64_t t1 = t0 + (int64_t)group_blocks * P < L ? t0 + (int64_t)group_blocks * P : L;
+        for (int h = 0; h < H; ++h) {
+            double *kh = khat + ((bg * H) + h) * D, *vh = vhat + ((bg * H) + h) * D;
+            for (int c = 0; c < D; ++c)
+                kh[c] = vh[c] = 0.0;
+            if (t1 <= t0)
+                continue;
+            for (int64_t tok = t0; tok < t1; ++tok) {
+                int64_t page = block_table[(int64_t)b * dm->max_blocks + tok / P];
+                for (int c = 0; c < D; ++c) {
+                    kh[c] += cache_at(dm, k_cache, k_scale, page, h, (int)(tok % P), c);
+                    vh[c] += cache_at(dm, v_cache, v_scale, page, h, (int)(tok % P), c);
+                }
+            }
+            for (int c = 0; c < D; ++c) {
+                kh[c] /= (double)(t1 - t0);
+                vh[c] /= (double)(t1 - t0);
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Dense attention of every query row over the pooled entries (§5.2: no
+ * selection).  Reading: entry g is visible to query token t when all its
+ * tokens are at or before the query's position L - Tq + t (no future token
+ * inside an entry); scale as the sparse branch; no position tag or sink logit
+ * (both need learned values).  out = softmax(q khat^T * scale) vhat; lse = ln
+ * of the sum of exp(logit) (-inf with no visible entry, out 0).
+ */
+int spo_hca_attend(const spo_dims *dm, const spo_params *pr, const uint16_t *q,
+                   const double *khat, const double *vhat, const int32_t *seq_lens,
+                   int group_blocks, double *out, double *lse)
+{
+    const int D = dm->head_dim, H = dm->num_kv_heads, Tq = dm->q_tokens;
+    const int P = dm->block_size, Hq = dm->num_q_heads, Gq = Hq / H;
+    const int Gmax = (dm->max_blocks + group_blocks - 1) / group_blocks;
+    const double scale = softmax_scale(dm, pr);
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t row = 0; row < (int64_t)dm->batch * Tq * Hq; ++row) {
+        int i = (int)(row % Hq), t = (int)((row / Hq) % Tq), b = (int)(row / ((int64_t)Hq * Tq));
+        int h = i / Gq;
+        int64_t L = seq_lens[b], qpos = L - Tq + t;
+        double *o = out + row * D;
+        const uint16_t *qr = q + row * D;
+        double *logit = (double *)malloc(sizeof(double) * (size_t)Gmax);
+        int n = 0;
+        for (int g = 0; g < Gmax; ++g) {
+            int64_t t0 = (int64_t)g * group_blocks * P;
+            int64_t last = t0 + (int64_t)group_blocks * P < L ? t0 + (int64_t)group_blocks * P - 1 : L - 1;
+            if (t0 >= L || last > qpos) break;
+            const double *kh = khat + (((int64_t)b * Gmax + g) * H + h) * D;
+            double dot = 0.0;
+            for (int c = 0; c < D; ++c)
+                dot += spo_bf16_to_f64(qr[c]) * kh[c];
+            logit[n++] = dot * scale;
+        }
+        for (int c = 0; c < D; ++c)
+            o[c] = 0.0;
+        lse[row] = -INFINITY;
+        if (n > 0) {
+            double mx = logit[0], z = 0.0;
+            for (int k = 1; k < n; ++k)
+                if (logit[k] > mx) mx = logit[k];
+            for (int k = 0; k < n; ++k)
+                z += exp(logit[k] - mx);
+            for (int k = 0; k < n; ++k) {
+                double p = exp(logit[k] - mx) / z;
+                const double *vh = vhat + (((int64_t)b * Gmax + k) * H + h) * D;
+                for (int c = 0; c < D; ++c)
+                    o[c] += p * vh[c];
+            }
+            lse[row] = mx + log(z);
+        }
+        free(logit);
     }
     return 0;
 }
