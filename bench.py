@@ -150,7 +150,21 @@ def step_bytes(inp, sel_count: torch.Tensor) -> dict:
     kbar = n_mid * H * D * (2 if w.kbar_bf16 else 4)
     q = inp["q"].numel() * 2
     out = inp["q"].numel() * 4
-    return dict(kv=kv, kbar=kbar, q=q, out=out, total=kv + kbar + q + out, kept_block_heads=kept)
+    d = dict(kv=kv, kbar=kbar, q=q, out=out, total=kv + kbar + q + out, kept_block_heads=kept)
+    if w.hca:
+        # HCA branch: the visible entries' K and V means (fp32, once per KV
+        # head), the appended tokens' entries re-pooled (their K and V read,
+        # two means written), and the branch outputs' round trip through the
+        # merge (HCA out written, both outputs read, the merged one written,
+        # three lse rows)
+        T, lens = 2 * P, inp["seq_lens"].tolist()
+        entries = sum((int(L) + T - 1) // T for L in lens)
+        pooled = sum(int(L) - (max(int(L) - w.q_tokens, 0) // T) * T for L in lens) * H * D * elt * 2
+        rows = inp["q"].numel() // D
+        attend = entries * H * D * 4 * 2 + 4 * out + 4 * rows * 4
+        hca = attend + pooled + len(lens) * H * D * 4 * 2
+        d.update(hca=hca, hca_attend=attend, total=d["total"] + hca)
+    return d
 
 
 def reduce_over_ranks(t: torch.Tensor, world: int) -> list:
@@ -211,6 +225,16 @@ def run_native(args, rank, world, local_rank):
 
     anchored = w.mode == "topp_anchor"   # the local blocks are scored: compress first
 
+    if w.hca:
+        # HCA branch: pooled entries (all of them now; the step re-pools the
+        # appended tokens' entries), its output / lse and the sparse lse
+        G = spattn.hca_entries(bt)
+        khat = torch.empty((B, G, Hkv, w.head_dim), dtype=torch.float32, device=dev)
+        vhat = torch.empty_like(khat)
+        spattn.hca_pool(kc, vc, ks, vs, bt, sl, khat, vhat)
+        lse_s = torch.empty(tuple(q.shape[:3]), dtype=torch.float32, device=dev)
+        out_s, o_hca, l_hca = torch.empty_like(out), torch.empty_like(out), torch.empty_like(lse_s)
+
     def front():   # scores + selection, with the tail block's compression beside them
         if anchored:
             spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
@@ -220,17 +244,28 @@ def run_native(args, rank, world, local_rank):
             with torch.cuda.stream(side):
                 spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
                                      q_tokens=Tq)
+                if w.hca:
+                    spattn.hca_pool(kc, vc, ks, vs, bt, sl, khat, vhat, old_lens=old_lens, q_tokens=Tq)
         spattn.block_scores(q, kbar, bt, sl, scores, params, k_cache=kc)
         spattn.select(scores, sl, sel_idx, sel_count, params, q=q, k_cache=kc, block_table=bt)
         if not anchored:
             torch.cuda.current_stream().wait_stream(side)
 
     def attend():  # sparse attention + split merge
-        spattn.decode_selected(q, kc, vc, ks, vs, bt, sl, sel_idx, sel_count, out, ws, params)
+        if not w.hca:
+            spattn.decode_selected(q, kc, vc, ks, vs, bt, sl, sel_idx, sel_count, out, ws, params)
+        else:
+            spattn.decode_selected(q, kc, vc, ks, vs, bt, sl, sel_idx, sel_count, out_s, ws, params, lse=lse_s)
+
+    def hca():     # the HCA branch's attention and the merge of the two branches
+        if w.hca:
+            spattn.hca_attend(q, khat, vhat, sl, o_hca, l_hca, params, k_cache=kc, block_table=bt)
+            spattn.lse_merge(out_s, lse_s, o_hca, l_hca, out)
 
     # warm up eagerly once (sets kernel attributes), then capture graphs
     front()
     attend()
+    hca()
     torch.cuda.synchronize()
     status = spattn.device_status()
     if status:
@@ -238,21 +273,31 @@ def run_native(args, rank, world, local_rank):
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        g_front, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        g_front, g_attn, g_hca = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_front, stream=s):
             front()
         with torch.cuda.graph(g_attn, stream=s):
             attend()
+        if w.hca:
+            with torch.cuda.graph(g_hca, stream=s):
+                hca()
+
+    def hca_replay():
+        if w.hca:
+            g_hca.replay()
     torch.cuda.current_stream().wait_stream(s)
     launches_per_step = 5          # compress, scores, select, attention, merge
+    if w.hca:
+        launches_per_step += 3     # hca_pool, hca_attend, lse_merge
 
     for _ in range(args.warmup):
         flush_l2()
         g_front.replay()
         g_attn.replay()
+        hca_replay()
     torch.cuda.synchronize()
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -271,12 +316,15 @@ def run_native(args, rank, world, local_rank):
             ev[i][1].record()
             g_attn.replay()
             ev[i][2].record()
+            hca_replay()
+            ev[i][3].record()
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     if world > 1:
         torch.distributed.barrier()
-    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    hca_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / K
     total_ms = sum(step_ms)
     bts = step_bytes(inp, sel_count)
     status = spattn.device_status()
@@ -295,6 +343,7 @@ def run_native(args, rank, world, local_rank):
         sl.copy_(sl_h, non_blocking=True)
         g_front.replay()
         g_attn.replay()
+        hca_replay()
         out_h.copy_(out, non_blocking=True)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
@@ -343,6 +392,11 @@ def run_native(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "wall_s": round(t_wall, 3),
     }
+    if w.hca:
+        line["hca"] = {"kernels": "hca_attend_kernel + lse_merge_kernel (one graph, timed apart from the sparse branch)",
+                       "ms_per_step": round(hca_ms, 5), "bytes": bts["hca_attend"],
+                       "achieved": round(bts["hca_attend"] / (hca_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                       "frac": round(bts["hca_attend"] / (hca_ms * 1e-3) / 1e9 / peak, 4)}
     if w.kbar_bf16:
         line["recall_vs_fp32_kbar"] = kbar_recall(inp, params, sel_idx, sel_count, dev)
     if world == 1:
@@ -394,19 +448,24 @@ def cpu_baseline(inp, bts, gpu_ms):
     ksc, vsc = sub["k_scale"].cpu().numpy(), sub["v_scale"].cpu().numpy()
     bt, sl = sub["block_table"].cpu().numpy(), sub["seq_lens"].cpu().numpy()
     kbar = oracle.compress_keys(dims, kh, ksc, bt, sl)
+    if w.hca:   # pooled entries, like the compressed keys, outside the timing
+        khat, vhat = oracle.hca_pool(dims, kh, vh, ksc, vsc, bt, sl)
     times = []
     t_end = time.perf_counter() + 10.0
     while time.perf_counter() < t_end or not times:
         t0 = time.perf_counter()
         sc = oracle.block_scores(dims, par, qh, kbar, bt, sl)
         sel, cnt, _ = oracle.select(dims, par, sc, sl)
-        oracle.attend(dims, par, qh, kh, vh, ksc, vsc, bt, sl, sel, cnt)
+        o_s = oracle.attend(dims, par, qh, kh, vh, ksc, vsc, bt, sl, sel, cnt, with_lse=w.hca)
+        if w.hca:
+            oracle.lse_merge(*o_s, *oracle.hca_attend(dims, par, qh, khat, vhat, sl))
         times.append(time.perf_counter() - t0)
     per_req = statistics.median(times)
     step_s = per_req * w.batch
     return {"value": round(bts["total"] / step_s / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"request 0 of {w.batch} (all {w.num_kv_heads} KV heads), {len(times)} runs, "
+            "sample": f"request 0 of {w.batch} (all {w.num_kv_heads} KV heads{', both branches' if w.hca else ''}), "
+                      f"{len(times)} runs, "
                       f"median {per_req:.3f} s, scaled x{w.batch} to the step",
             "ms_per_step": round(step_s * 1e3, 3), "gpu_speedup": round(step_s * 1e3 / gpu_ms, 1)}
 
@@ -432,14 +491,21 @@ def run_reference(args, rank, world):
         ksc, vsc = sub["k_scale"].cpu().numpy(), sub["v_scale"].cpu().numpy()
         bt, sl = sub["block_table"].cpu().numpy(), sub["seq_lens"].cpu().numpy()
         kbar = oracle.compress_keys(dims, kh, ksc, bt, sl)
-        subs.append((dims, qh, kh, vh, ksc, vsc, bt, sl, kbar))
-    units = w.batch * w.num_kv_heads
+        hat = oracle.hca_pool(dims, kh, vh, ksc, vsc, bt, sl) if w.hca else None
+        subs.append((dims, qh, kh, vh, ksc, vsc, bt, sl, kbar, hat))
+    # with the HCA branch a unit is a whole request (its dense attention
+    # covers all KV heads at once); otherwise one (request, KV head)
+    units = w.batch * (1 if w.hca else w.num_kv_heads)
 
     def one(i):
-        dims, qh, kh, vh, ksc, vsc, bt, sl, kbar = subs[i % len(subs)]
-        h = (i // len(subs)) % w.num_kv_heads
+        dims, qh, kh, vh, ksc, vsc, bt, sl, kbar, hat = subs[i % len(subs)]
         sc = oracle.block_scores(dims, par, qh, kbar, bt, sl)
         sel, cnt, _ = oracle.select(dims, par, sc, sl)
+        if w.hca:
+            o_s = oracle.attend(dims, par, qh, kh, vh, ksc, vsc, bt, sl, sel, cnt, with_lse=True)
+            oracle.lse_merge(*o_s, *oracle.hca_attend(dims, par, qh, hat[0], hat[1], sl))
+            return int(cnt[0].sum())
+        h = (i // len(subs)) % w.num_kv_heads
         oracle.attend(dims, par, qh, kh, vh, ksc, vsc, bt, sl, sel, cnt, units=[(0, h)])
         return int(cnt[0, h])
 
@@ -462,9 +528,12 @@ def run_reference(args, rank, world):
     nbs = [(int(L) + P - 1) // P for L in inp["seq_lens"].tolist()]
     n_mid = sum(max(0, nb - w.sink_blocks - w.local_blocks) for nb in nbs)
     total = units * mean_kept * P * D * elt * 2 + n_mid * w.num_kv_heads * D * 4 + inp["q"].numel() * 6
+    if w.hca:
+        total += step_bytes(inp, torch.zeros(1))["hca"]
     value = total / step_s / 1e9
-    sample = (f"{len(times)} steps x one (request, KV head) unit of {units} (scores, selection, attention "
-              f"in float64), scaled x{units} to the step")
+    what = "request" if w.hca else "(request, KV head)"
+    sample = (f"{len(times)} steps x one {what} unit of {units} (scores, selection, attention"
+              f"{', HCA branch and merge' if w.hca else ''} in float64), scaled x{units} to the step")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
         "n_gpus": world, "steps": len(times), "warmup": args.warmup,

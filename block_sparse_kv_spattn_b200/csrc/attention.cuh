@@ -515,6 +515,7 @@ struct MergeArgs {
     const float *part_ml;
     const int32_t *sel_count;
     float *out;                 // [B][Tq][Hq][D]
+    float *lse;                 // nullable: [B][Tq][Hq], ln of the row's sum of exp(logit)
     int batch, tq, hq, hkv, group, rows, units, max_sel, ctas;
     int wslots;                 // partial records per (CTA, unit): 1, or one per tensor-core softmax warp
 };
@@ -628,6 +629,7 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
         if (warp != 0) return;
         float Mt = -INFINITY;
         for (int w = 0; w < nw; ++w) Mt = fmaxf(Mt, s_m[w]);
+        M = Mt;
         acc = make_float4(0.f, 0.f, 0.f, 0.f);
         lsum = 0.f;
         if (Mt != -INFINITY)
@@ -645,6 +647,8 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
     reinterpret_cast<float4 *>(a.out + grow * kHeadDim)[lane] =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    // records hold base-2 maxima of the scaled logits: ln sum = (M + log2 l) ln 2
+    if (a.lse && lane == 0) a.lse[grow] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace spattn

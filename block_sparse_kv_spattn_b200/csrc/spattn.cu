@@ -21,6 +21,7 @@
 #include "select.cuh"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "hca.cuh"
 
 using namespace spattn;
 
@@ -426,7 +427,7 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
                                const void *k_cache, const void *v_cache, const float *k_scale,
                                const float *v_scale, const int32_t *bt, const int32_t *sl,
                                const int32_t *sel_idx, const int32_t *sel_count, float *out,
-                               char *ws, const DecodeLayout &L, cudaStream_t st) {
+                               float *lse, char *ws, const DecodeLayout &L, cudaStream_t st) {
     const bool fp8 = d->kv_dtype == SPATTN_KV_FP8_E4M3;
     const int rows = rows_of(d);
     const int rg = rg_of(rows);
@@ -466,6 +467,7 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.part_ml = a.part_ml;
     m.sel_count = sel_count;
     m.out = out;
+    m.lse = lse;
     m.batch = d->batch;
     m.tq = d->q_tokens;
     m.hq = d->num_q_heads;
@@ -628,6 +630,16 @@ spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_param
                                      const int32_t *seq_lens, const int32_t *sel_idx,
                                      const int32_t *sel_count, float *out, void *workspace,
                                      size_t workspace_bytes, spattn_stream_t stream) {
+    return spattn_decode_selected_lse(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
+                                      sel_idx, sel_count, out, nullptr, workspace, workspace_bytes, stream);
+}
+
+spattn_status spattn_decode_selected_lse(const spattn_dims *dims, const spattn_params *params, const void *q,
+                                         const void *k_cache, const void *v_cache, const float *k_scale,
+                                         const float *v_scale, const int32_t *block_table,
+                                         const int32_t *seq_lens, const int32_t *sel_idx,
+                                         const int32_t *sel_count, float *out, float *lse, void *workspace,
+                                         size_t workspace_bytes, spattn_stream_t stream) {
     SP_TRY(check_dims(dims));
     SP_TRY(check_params(params));
     SP_TRY(check_cache_args(dims, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens));
@@ -641,7 +653,7 @@ spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_param
         return fail(SPATTN_ERR_WORKSPACE, "workspace must be %zu-byte aligned", kAlign);
     char *ws = static_cast<char *>(workspace);
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
-                            sel_idx, sel_count, out, ws, L, reinterpret_cast<cudaStream_t>(stream)));
+                            sel_idx, sel_count, out, lse, ws, L, reinterpret_cast<cudaStream_t>(stream)));
     return ok();
 }
 
@@ -667,7 +679,7 @@ spattn_status spattn_decode_selected_noalloc(const spattn_dims *dims, const spat
     SP_TRY(noalloc_scratch(&scratch));
     char *ws = static_cast<char *>(scratch);
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
-                            sel_idx, sel_count, out, ws, L, reinterpret_cast<cudaStream_t>(stream)));
+                            sel_idx, sel_count, out, nullptr, ws, L, reinterpret_cast<cudaStream_t>(stream)));
     return ok();
 }
 
@@ -698,7 +710,101 @@ spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params
     SP_TRY(launch_scores(dims, params, q, kbar, block_table, seq_lens, scores, st));
     SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count, st));
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
-                            sel_idx, sel_count, out, ws, L, st));
+                            sel_idx, sel_count, out, nullptr, ws, L, st));
+    return ok();
+}
+
+// ---------------------------------------------------------------- HCA branch
+
+int32_t spattn_hca_entries(const spattn_dims *dims) {
+    if (check_dims(dims) != SPATTN_OK) return -1;
+    return (dims->max_blocks_per_seq + kHcaGroupBlocks - 1) / kHcaGroupBlocks;
+}
+
+spattn_status spattn_hca_pool(const spattn_dims *dims, const void *k_cache, const void *v_cache,
+                              const float *k_scale, const float *v_scale, const int32_t *block_table,
+                              const int32_t *old_lens, const int32_t *seq_lens, float *khat, float *vhat,
+                              spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    if (!k_cache || !v_cache || !block_table || !seq_lens || !khat || !vhat)
+        return fail(SPATTN_ERR_INVALID_ARG, "k_cache, v_cache, block_table, seq_lens, khat, vhat are required");
+    const bool fp8 = dims->kv_dtype == SPATTN_KV_FP8_E4M3;
+    if (fp8 && (!k_scale || !v_scale)) return fail(SPATTN_ERR_INVALID_ARG, "fp8 caches need k_scale and v_scale");
+    if (((uintptr_t)k_cache | (uintptr_t)v_cache | (uintptr_t)khat | (uintptr_t)vhat) & 15)
+        return fail(SPATTN_ERR_INVALID_ARG, "k_cache, v_cache, khat and vhat must be 16-byte aligned");
+    HcaPoolArgs a;
+    a.k_cache = static_cast<const uint8_t *>(k_cache);
+    a.v_cache = static_cast<const uint8_t *>(v_cache);
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.block_table = block_table;
+    a.old_lens = old_lens;
+    a.seq_lens = seq_lens;
+    a.khat = khat;
+    a.vhat = vhat;
+    a.hkv = dims->num_kv_heads;
+    a.num_pages = dims->num_pages;
+    a.max_blocks = dims->max_blocks_per_seq;
+    a.gmax = spattn_hca_entries(dims);
+    // incremental: the entries of the appended tokens (q_tokens of them, the
+    // CTAs stride over more if a request grew further)
+    const int gx = old_lens ? (dims->q_tokens + kHcaTokens - 1) / kHcaTokens + 1 : a.gmax;
+    const dim3 grid(gx, dims->batch), block(32 * dims->num_kv_heads);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (fp8)
+        hca_pool_kernel<true><<<grid, block, 0, st>>>(a);
+    else
+        hca_pool_kernel<false><<<grid, block, 0, st>>>(a);
+    SP_TRY(cuda_ok(cudaGetLastError(), "hca_pool launch"));
+    return ok();
+}
+
+spattn_status spattn_hca_attend(const spattn_dims *dims, const spattn_params *params, const void *q,
+                                const float *khat, const float *vhat, const int32_t *seq_lens, float *out,
+                                float *lse, spattn_stream_t stream) {
+    SP_TRY(check_dims(dims));
+    SP_TRY(check_params(params));
+    if (!q || !khat || !vhat || !seq_lens || !out || !lse)
+        return fail(SPATTN_ERR_INVALID_ARG, "q, khat, vhat, seq_lens, out, lse are required");
+    if (((uintptr_t)q | (uintptr_t)khat | (uintptr_t)vhat | (uintptr_t)out) & 15)
+        return fail(SPATTN_ERR_INVALID_ARG, "q, khat, vhat and out must be 16-byte aligned");
+    HcaAttendArgs a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.khat = khat;
+    a.vhat = vhat;
+    a.seq_lens = seq_lens;
+    a.out = out;
+    a.lse = lse;
+    a.tq = dims->q_tokens;
+    a.hq = dims->num_q_heads;
+    a.hkv = dims->num_kv_heads;
+    a.max_blocks = dims->max_blocks_per_seq;
+    a.gmax = spattn_hca_entries(dims);
+    a.qscale = sm_scale_of(params) * kLog2e;
+    const int64_t rows = (int64_t)dims->batch * dims->q_tokens * dims->num_q_heads;
+    SP_TRY(cuda_ok(launch(hca_attend_kernel, dim3((unsigned)rows), dim3(32 * kHcaWarps), 0,
+                          reinterpret_cast<cudaStream_t>(stream), a),
+                   "hca_attend launch"));
+    return ok();
+}
+
+spattn_status spattn_lse_merge(const spattn_dims *dims, const float *out_a, const float *lse_a,
+                               const float *out_b, const float *lse_b, float *out, float *lse,
+                               spattn_stream_t stream) {
+    // only the row count and d matter here
+    if (!dims) return fail(SPATTN_ERR_INVALID_ARG, "dims is NULL");
+    if (dims->batch < 1 || dims->q_tokens < 1 || dims->num_q_heads < 1)
+        return fail(SPATTN_ERR_INVALID_ARG, "dims: batch, q_tokens, num_q_heads must be positive");
+    if (dims->head_dim != kHeadDim)
+        return fail(SPATTN_ERR_UNSUPPORTED, "head_dim %d: only %d is built", dims->head_dim, kHeadDim);
+    if (!out_a || !lse_a || !out_b || !lse_b || !out)
+        return fail(SPATTN_ERR_INVALID_ARG, "out_a, lse_a, out_b, lse_b, out are required");
+    if (((uintptr_t)out_a | (uintptr_t)out_b | (uintptr_t)out) & 15)
+        return fail(SPATTN_ERR_INVALID_ARG, "out_a, out_b and out must be 16-byte aligned");
+    const int64_t rows = (int64_t)dims->batch * dims->q_tokens * dims->num_q_heads;
+    SP_TRY(cuda_ok(launch(lse_merge_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0,
+                          reinterpret_cast<cudaStream_t>(stream), rows, out_a, lse_a, out_b, lse_b, out, lse),
+                   "lse_merge launch"));
     return ok();
 }
 

@@ -10,7 +10,8 @@ Layouts are those of the header: q bf16 [B][Tq][Hq][128]; caches bf16 (or
 uint8 e4m3fn codes) [num_pages][Hkv][64][128]; scales f32 [num_pages][Hkv];
 block_table int32 [B][max_blocks]; seq_lens int32 [B]; kbar f32
 [num_pages][Hkv][128]; scores f32 [B][Tq][Hkv][max_blocks]; sel_idx int32
-[B][Hkv][max_sel]; sel_count int32 [B][Hkv]; out f32 [B][Tq][Hq][128].
+[B][Hkv][max_sel]; sel_count int32 [B][Hkv]; out f32 [B][Tq][Hq][128];
+lse f32 [B][Tq][Hq]; khat / vhat f32 [B][ceil(max_blocks / 2)][Hkv][128].
 """
 from __future__ import annotations
 
@@ -36,7 +37,8 @@ KBAR_F32, KBAR_BF16 = 0, 1
 EXPORTS = ("spattn_required_max_sel", "spattn_compress_keys", "spattn_block_scores",
            "spattn_select", "spattn_decode_workspace_size", "spattn_decode_selected",
            "spattn_decode", "spattn_last_error", "spattn_get_device_status", "spattn_version",
-           "spattn_decode_selected_noalloc")
+           "spattn_decode_selected_noalloc", "spattn_decode_selected_lse", "spattn_hca_entries",
+           "spattn_hca_pool", "spattn_hca_attend", "spattn_lse_merge")
 
 
 class SpattnError(RuntimeError):
@@ -100,6 +102,11 @@ def load() -> ctypes.CDLL:
         "spattn_get_device_status": ([P, P], ctypes.c_int),
         "spattn_version": ([], ctypes.c_char_p),
         "spattn_decode_selected_noalloc": ([P] * 13, ctypes.c_int),
+        "spattn_decode_selected_lse": ([P] * 14 + [ctypes.c_size_t, P], ctypes.c_int),
+        "spattn_hca_entries": ([P], I32),
+        "spattn_hca_pool": ([P] * 11, ctypes.c_int),
+        "spattn_hca_attend": ([P] * 9, ctypes.c_int),
+        "spattn_lse_merge": ([P] * 8, ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -186,14 +193,19 @@ def select(scores, seq_lens, sel_idx, sel_count, params: Params, *, q, k_cache, 
 
 
 def decode_selected(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, sel_idx,
-                    sel_count, out, workspace, params: Params, stream=None):
+                    sel_count, out, workspace, params: Params, stream=None, lse=None):
+    """Attention over the given selection; with ``lse`` (f32 [B][Tq][Hq])
+    also each row's log-sum-exp (spattn_decode_selected_lse)."""
     dims = dims_for(q, k_cache, block_table, sel_idx.shape[-1])
     fp8 = dims.kv_dtype == KV_FP8_E4M3
-    _check(load().spattn_decode_selected(
-        ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(k_cache), _p(v_cache),
-        _p(k_scale) if fp8 else None, _p(v_scale) if fp8 else None, _p(block_table),
-        _p(seq_lens), _p(sel_idx), _p(sel_count), _p(out), _p(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)))
+    args = [ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(k_cache), _p(v_cache),
+            _p(k_scale) if fp8 else None, _p(v_scale) if fp8 else None, _p(block_table),
+            _p(seq_lens), _p(sel_idx), _p(sel_count), _p(out)]
+    tail = [_p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)]
+    if lse is None:
+        _check(load().spattn_decode_selected(*args, *tail))
+    else:
+        _check(load().spattn_decode_selected_lse(*args, _p(lse), *tail))
 
 
 def decode_selected_noalloc(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, sel_idx,
@@ -217,6 +229,46 @@ def decode(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, kbar, o
         _p(k_scale) if fp8 else None, _p(v_scale) if fp8 else None, _p(block_table),
         _p(seq_lens), _p(kbar), _p(out), _p(sel_idx), _p(sel_count), _p(scores_out),
         _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ------------------------------------------------------------------ HCA branch
+
+HCA_BLOCKS = 2      # blocks per pooled entry (128 tokens)
+
+
+def hca_entries(block_table) -> int:
+    """Entries per request of the khat / vhat buffers."""
+    return (block_table.shape[1] + HCA_BLOCKS - 1) // HCA_BLOCKS
+
+
+def hca_pool(k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, khat, vhat, old_lens=None, *,
+             q_tokens: int = 1, stream=None):
+    """Mean K and V of every 128-token entry: khat / vhat f32 [B][G][Hkv][128]."""
+    num_pages, Hkv, P, D = k_cache.shape
+    kv = KV_FP8_E4M3 if k_cache.dtype in (torch.uint8, torch.float8_e4m3fn) else KV_BF16
+    dims = CDims(seq_lens.shape[0], q_tokens, Hkv, Hkv, D, P, num_pages, block_table.shape[1], 0, kv,
+                 KBAR_F32)
+    fp8 = kv == KV_FP8_E4M3
+    _check(load().spattn_hca_pool(ctypes.byref(dims), _p(k_cache), _p(v_cache),
+                                  _p(k_scale) if fp8 else None, _p(v_scale) if fp8 else None,
+                                  _p(block_table), _p(old_lens), _p(seq_lens), _p(khat), _p(vhat),
+                                  _stream(stream)))
+
+
+def hca_attend(q, khat, vhat, seq_lens, out, lse, params: Params, *, k_cache, block_table, stream=None):
+    """Dense attention of every query row over its visible pooled entries."""
+    dims = dims_for(q, k_cache, block_table)
+    _check(load().spattn_hca_attend(ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(khat), _p(vhat),
+                                    _p(seq_lens), _p(out), _p(lse), _stream(stream)))
+
+
+def lse_merge(out_a, lse_a, out_b, lse_b, out, lse=None, stream=None):
+    """One softmax over two disjoint key sets from two partial results
+    ([B][Tq][Hq][128] outputs, [B][Tq][Hq] log-sum-exps)."""
+    B, Tq, Hq, D = out_a.shape
+    dims = CDims(B, Tq, Hq, 1, D, 64, 1, 1, 0, KV_BF16, KBAR_F32)
+    _check(load().spattn_lse_merge(ctypes.byref(dims), _p(out_a), _p(lse_a), _p(out_b), _p(lse_b), _p(out),
+                                   _p(lse), _stream(stream)))
 
 
 def device_status(stream=None) -> int:

@@ -55,6 +55,7 @@ class Workload:
     max_ratio: float = 0.0
     min_ratio: float = 0.0            # topp_anchor: the cap ratio when the anchors dominate
     kbar_bf16: bool = False           # compressed keys stored as bf16 (low-precision scoring)
+    hca: bool = False                 # add the dense branch over 128-token mean entries
     sink_blocks: int = 1
     local_blocks: int = 2
     head_dim: int = HEAD_DIM
@@ -87,6 +88,11 @@ WORKLOADS = {
     "decode_128k_b8_kbar16": Workload("decode_128k_b8_kbar16", batch=8, q_tokens=1, num_q_heads=32,
                                       num_kv_heads=8, seq_len=131072, structure="zipf", mode="topp",
                                       top_p=0.9, max_ratio=0.15, kbar_bf16=True, seed=1236),
+    # the gate shape with the weight-free HCA branch beside the sparse one
+    # (pooled 128-token entries, dense attention, log-sum-exp merge)
+    "decode_128k_b8_hca": Workload("decode_128k_b8_hca", batch=8, q_tokens=1, num_q_heads=32,
+                                   num_kv_heads=8, seq_len=131072, structure="zipf", mode="topp",
+                                   top_p=0.9, max_ratio=0.15, hca=True, seed=1236),
     # the same shape with 2 requests: small enough for detailed profiling
     "decode_128k_b2": Workload("decode_128k_b2", batch=2, q_tokens=1, num_q_heads=32, num_kv_heads=8,
                                seq_len=131072, structure="zipf", mode="topp", top_p=0.9,

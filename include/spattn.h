@@ -231,6 +231,25 @@ spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_param
                                      spattn_stream_t stream);
 
 /*
+ * spattn_decode_selected_lse -- spattn_decode_selected that also reports each
+ * row's log-sum-exp, so that its result can be combined with another
+ * branch's over a disjoint key set ("CSA + HCA 混合注意力机制" §6: the sparse
+ * and the compressed branches joined into one softmax).
+ *
+ * lse (device, fp32 [B][Tq][Hq], may be NULL = spattn_decode_selected)
+ * receives ln(sum over the row's visible kept tokens of
+ * exp(sm_scale * q . k_tau)), -inf for a row with no visible token.
+ * Everything else as spattn_decode_selected.
+ */
+spattn_status spattn_decode_selected_lse(const spattn_dims *dims, const spattn_params *params,
+                                         const void *q, const void *k_cache, const void *v_cache,
+                                         const float *k_scale, const float *v_scale,
+                                         const int32_t *block_table, const int32_t *seq_lens,
+                                         const int32_t *sel_idx, const int32_t *sel_count,
+                                         float *out, float *lse, void *workspace,
+                                         size_t workspace_bytes, spattn_stream_t stream);
+
+/*
  * spattn_decode_selected_noalloc -- spattn_decode_selected without a
  * caller-supplied workspace.  (Not a step of the method: the pages have no
  * counterpart; it only changes where the scratch memory lives.)
@@ -277,6 +296,71 @@ spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params
                             const void *kbar, float *out, int32_t *sel_idx,
                             int32_t *sel_count, float *scores_out, void *workspace,
                             size_t workspace_bytes, spattn_stream_t stream);
+
+/* ================================================================ HCA branch
+ *
+ * The weight-free compressed branch ("CSA + HCA 混合注意力机制" §5.1-5.2): every
+ * SPATTN_HCA_BLOCKS consecutive blocks (m' = 128 tokens) of a request are
+ * pooled into one key entry and one value entry, and every query attends
+ * densely over its request's visible entries (no selection).  Readings of
+ * the page: the page's learned pooling is replaced by the mean over the
+ * entry's filled tokens; an entry is visible to query token t when all its
+ * tokens are at or before position seq_lens[b] - Tq + t; no position tag
+ * and no learned sink logit.  The branch's output joins the sparse branch's
+ * (spattn_decode_selected_lse) through spattn_lse_merge, which is softmax
+ * attention over the union of both key sets.
+ *
+ * khat / vhat are device fp32 [B][G][Hkv][d] with G = spattn_hca_entries().
+ */
+#define SPATTN_HCA_BLOCKS 2
+
+/* G = ceil(max_blocks_per_seq / SPATTN_HCA_BLOCKS): entries per request in
+ * the khat / vhat buffers.  Returns -1 on invalid dims. */
+int32_t spattn_hca_entries(const spattn_dims *dims);
+
+/*
+ * spattn_hca_pool -- mean K and V of each entry.
+ *
+ * khat[b][g][h][:] = mean over the tokens [128 g, min(L, 128 (g + 1))) of
+ * request b of K (dequantised with k_scale for fp8; fp32 sums), vhat the same
+ * of V.  With old_lens == NULL every entry of every request is written
+ * (entries past the end of a request: zeros); otherwise only the entries
+ * that hold a token of [old_lens[b], seq_lens[b]).  k_scale / v_scale may be
+ * NULL for bf16 caches.  Block-table entries outside the pool are skipped
+ * and set SPATTN_DEV_BAD_PAGE; a bad seq_len sets SPATTN_DEV_BAD_LEN.
+ */
+spattn_status spattn_hca_pool(const spattn_dims *dims, const void *k_cache, const void *v_cache,
+                              const float *k_scale, const float *v_scale,
+                              const int32_t *block_table, const int32_t *old_lens,
+                              const int32_t *seq_lens, float *khat, float *vhat,
+                              spattn_stream_t stream);
+
+/*
+ * spattn_hca_attend -- dense attention over the pooled entries.
+ *
+ * out[b][t][i][:] = softmax_g(sm_scale * q . khat[b][g][h]) vhat[b][g][h]
+ * over the visible entries g of (b, t), h = i / (Hq / Hkv); lse[b][t][i] =
+ * ln of the softmax's denominator.  A row with no visible entry gets zeros
+ * and -inf.  fp32 throughout; out and lse are device [B][Tq][Hq][d] and
+ * [B][Tq][Hq] (both required).
+ */
+spattn_status spattn_hca_attend(const spattn_dims *dims, const spattn_params *params,
+                                const void *q, const float *khat, const float *vhat,
+                                const int32_t *seq_lens, float *out, float *lse,
+                                spattn_stream_t stream);
+
+/*
+ * spattn_lse_merge -- one softmax over two disjoint key sets from the two
+ * partial results (B * Tq * Hq rows of d):
+ *   out = (e^lse_a out_a + e^lse_b out_b) / (e^lse_a + e^lse_b),
+ *   lse = ln(e^lse_a + e^lse_b)   (lse may be NULL).
+ * A row whose two lse are -inf gets zeros and -inf.  out / lse may be the
+ * same buffers as out_a / lse_a or out_b / lse_b.  Device fp32 pointers.
+ * Of dims only batch, q_tokens, num_q_heads and head_dim (128) are read.
+ */
+spattn_status spattn_lse_merge(const spattn_dims *dims, const float *out_a, const float *lse_a,
+                               const float *out_b, const float *lse_b, float *out, float *lse,
+                               spattn_stream_t stream);
 
 /* Message for the last failed call on this host thread ("" if none). */
 const char *spattn_last_error(void);

@@ -105,3 +105,30 @@ def test_small_max_sel_and_workspace_rejected(lib):
 
 def test_version(lib):
     assert "sm_100a" in spattn.version()
+
+
+def test_hca_entry_points_validate_on_the_host(lib):
+    """The HCA entries and the lse variant check sizes, pointers and
+    alignment before enqueueing anything."""
+    d, p = _dims(max_blocks_per_seq=51), spattn.Params(top_k=4)
+    dummy, odd = ctypes.c_void_p(256), ctypes.c_void_p(260)
+    assert lib.spattn_hca_entries(ctypes.byref(d)) == 26          # ceil(51 / 2)
+    assert lib.spattn_hca_entries(ctypes.byref(_dims(head_dim=64))) == -1
+    assert lib.spattn_hca_pool(ctypes.byref(d), dummy, dummy, None, None, dummy, None, dummy, None, dummy,
+                               None) == 1
+    d.kv_dtype = 1
+    assert lib.spattn_hca_pool(ctypes.byref(d), dummy, dummy, None, None, dummy, None, dummy, dummy, dummy,
+                               None) == 1
+    assert b"scale" in lib.spattn_last_error()
+    d.kv_dtype = 0
+    assert lib.spattn_hca_pool(ctypes.byref(d), dummy, dummy, None, None, dummy, None, dummy, odd, dummy,
+                               None) == 1
+    assert b"aligned" in lib.spattn_last_error()
+    assert lib.spattn_hca_attend(ctypes.byref(d), ctypes.byref(p.c()), dummy, dummy, dummy, dummy, dummy,
+                                 None, None) == 1
+    assert lib.spattn_lse_merge(ctypes.byref(d), dummy, dummy, dummy, None, dummy, None, None) == 1
+    assert lib.spattn_lse_merge(ctypes.byref(_dims(head_dim=96)), dummy, dummy, dummy, dummy, dummy, None,
+                                None) == 2
+    st = lib.spattn_decode_selected_lse(ctypes.byref(d), ctypes.byref(p.c()), dummy, dummy, dummy, None,
+                                        None, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 16, None)
+    assert st == 4
