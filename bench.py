@@ -154,14 +154,14 @@ def step_bytes(inp, sel_count: torch.Tensor) -> dict:
     if w.hca:
         # HCA branch: the visible entries' K and V means (fp32, once per KV
         # head), the appended tokens' entries re-pooled (their K and V read,
-        # two means written), and the branch outputs' round trip through the
-        # merge (HCA out written, both outputs read, the merged one written,
-        # three lse rows)
+        # two means written), and the sparse branch's result read back into
+        # the merged output (its out read, the merged out written, its lse
+        # written and read)
         T, lens = 2 * P, inp["seq_lens"].tolist()
         entries = sum((int(L) + T - 1) // T for L in lens)
         pooled = sum(int(L) - (max(int(L) - w.q_tokens, 0) // T) * T for L in lens) * H * D * elt * 2
         rows = inp["q"].numel() // D
-        attend = entries * H * D * 4 * 2 + 4 * out + 4 * rows * 4
+        attend = entries * H * D * 4 * 2 + 2 * out + 2 * rows * 4
         hca = attend + pooled + len(lens) * H * D * 4 * 2
         d.update(hca=hca, hca_attend=attend, total=d["total"] + hca)
     return d
@@ -229,11 +229,12 @@ def run_native(args, rank, world, local_rank):
         # HCA branch: pooled entries (all of them now; the step re-pools the
         # appended tokens' entries), its output / lse and the sparse lse
         G = spattn.hca_entries(bt)
-        khat = torch.empty((B, G, Hkv, w.head_dim), dtype=torch.float32, device=dev)
+        khat = torch.empty((B, Hkv, G, w.head_dim), dtype=torch.float32, device=dev)
         vhat = torch.empty_like(khat)
         spattn.hca_pool(kc, vc, ks, vs, bt, sl, khat, vhat)
         lse_s = torch.empty(tuple(q.shape[:3]), dtype=torch.float32, device=dev)
-        out_s, o_hca, l_hca = torch.empty_like(out), torch.empty_like(out), torch.empty_like(lse_s)
+        out_s = torch.empty_like(out)
+        hca_ws = spattn.hca_workspace(q, kc, bt)
 
     def front():   # scores + selection, with the tail block's compression beside them
         if anchored:
@@ -259,8 +260,8 @@ def run_native(args, rank, world, local_rank):
 
     def hca():     # the HCA branch's attention and the merge of the two branches
         if w.hca:
-            spattn.hca_attend(q, khat, vhat, sl, o_hca, l_hca, params, k_cache=kc, block_table=bt)
-            spattn.lse_merge(out_s, lse_s, o_hca, l_hca, out)
+            spattn.hca_attend(q, khat, vhat, sl, out, None, params, k_cache=kc, block_table=bt, workspace=hca_ws,
+                              merge_with=(out_s, lse_s))
 
     # warm up eagerly once (sets kernel attributes), then capture graphs
     front()
@@ -288,7 +289,7 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.current_stream().wait_stream(s)
     launches_per_step = 5          # compress, scores, select, attention, merge
     if w.hca:
-        launches_per_step += 3     # hca_pool, hca_attend, lse_merge
+        launches_per_step += 3     # hca_pool, hca_partial, hca_combine (merging the sparse result)
 
     for _ in range(args.warmup):
         flush_l2()
@@ -393,7 +394,8 @@ def run_native(args, rank, world, local_rank):
         "wall_s": round(t_wall, 3),
     }
     if w.hca:
-        line["hca"] = {"kernels": "hca_attend_kernel + lse_merge_kernel (one graph, timed apart from the sparse branch)",
+        line["hca"] = {"kernels": "hca_partial_kernel + hca_combine_kernel merging the sparse result "
+                                  "(timed apart from the sparse branch)",
                        "ms_per_step": round(hca_ms, 5), "bytes": bts["hca_attend"],
                        "achieved": round(bts["hca_attend"] / (hca_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                        "frac": round(bts["hca_attend"] / (hca_ms * 1e-3) / 1e9 / peak, 4)}

@@ -542,6 +542,80 @@ constexpr bool tc_layout_ok() {
 static_assert(tc_layout_ok<4>() && tc_layout_ok<8>() && tc_layout_ok<16>(),
               "one CTA per SM; even stage count; swizzled operand tiles on 1024-byte boundaries");
 
+// Split of the HCA attention: CTAs per (request, KV head), so that all
+// CTAs fit in one wave at two per SM.
+int hca_split(int units, int sms) {
+    const int s = 2 * sms / units;
+    return s < 1 ? 1 : (s > kHcaMaxSplit ? kHcaMaxSplit : s);
+}
+
+size_t hca_workspace_bytes(const spattn_dims *d) {
+    const size_t recs = (size_t)d->batch * d->num_kv_heads * kHcaMaxSplit * rows_of(d);
+    return align_up(recs * kHeadDim * 4) + align_up(recs * 2 * 4);
+}
+
+// The HCA branch's attention (optionally merged with another branch's
+// result): partial records per share of the entries, then their merge.
+spattn_status launch_hca_attend(const spattn_dims *d, const spattn_params *p, const void *q, const float *khat,
+                                const float *vhat, const int32_t *sl, const float *base_out,
+                                const float *base_lse, float *out, float *lse, void *workspace,
+                                size_t workspace_bytes, cudaStream_t st) {
+    SP_TRY(check_dims(d));
+    SP_TRY(check_params(p));
+    if (!q || !khat || !vhat || !sl || !out)
+        return fail(SPATTN_ERR_INVALID_ARG, "q, khat, vhat, seq_lens, out are required");
+    if (((uintptr_t)q | (uintptr_t)khat | (uintptr_t)vhat | (uintptr_t)out) & 15)
+        return fail(SPATTN_ERR_INVALID_ARG, "q, khat, vhat and out must be 16-byte aligned");
+    const size_t need = hca_workspace_bytes(d);
+    if (!workspace || workspace_bytes < need)
+        return fail(SPATTN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
+    if ((uintptr_t)workspace & (kAlign - 1))
+        return fail(SPATTN_ERR_WORKSPACE, "workspace must be %zu-byte aligned", kAlign);
+    int sms;
+    SP_TRY(sm_count(&sms));
+    const int units = d->batch * d->num_kv_heads;
+    const size_t recs = (size_t)units * kHcaMaxSplit * rows_of(d);
+    HcaAttendArgs a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.khat = khat;
+    a.vhat = vhat;
+    a.seq_lens = sl;
+    a.part_o = static_cast<float *>(workspace);
+    a.part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) + align_up(recs * kHeadDim * 4));
+    a.tq = d->q_tokens;
+    a.hq = d->num_q_heads;
+    a.hkv = d->num_kv_heads;
+    a.max_blocks = d->max_blocks_per_seq;
+    a.gmax = (d->max_blocks_per_seq + kHcaGroupBlocks - 1) / kHcaGroupBlocks;
+    a.split = hca_split(units, sms);
+    a.qscale = sm_scale_of(p) * kLog2e;
+    const dim3 grid(a.split, units), block(32 * (kHcaCtaWarps + 1));
+    cudaError_t e;
+    if (rows_of(d) <= 4) {
+        SP_TRY(ensure_smem((const void *)hca_partial_kernel<4, 8>, HcaRing<8>::kSmem));
+        e = launch(hca_partial_kernel<4, 8>, grid, block, HcaRing<8>::kSmem, st, a);
+    } else {
+        SP_TRY(ensure_smem((const void *)hca_partial_kernel<8, 4>, HcaRing<4>::kSmem));
+        e = launch(hca_partial_kernel<8, 4>, grid, block, HcaRing<4>::kSmem, st, a);
+    }
+    SP_TRY(cuda_ok(e, "hca_partial launch"));
+    HcaCombineArgs c;
+    c.part_o = a.part_o;
+    c.part_ml = a.part_ml;
+    c.base_out = base_out;
+    c.base_lse = base_lse;
+    c.out = out;
+    c.lse = lse;
+    c.nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
+    c.tq = d->q_tokens;
+    c.hq = d->num_q_heads;
+    c.hkv = d->num_kv_heads;
+    c.split = a.split;
+    SP_TRY(cuda_ok(launch(hca_combine_kernel, dim3((unsigned)((c.nrows + 7) / 8)), dim3(256), 0, st, c),
+                   "hca_combine launch"));
+    return ok();
+}
+
 }  // namespace
 
 // ================================================================ C ABI
@@ -759,33 +833,27 @@ spattn_status spattn_hca_pool(const spattn_dims *dims, const void *k_cache, cons
     return ok();
 }
 
+size_t spattn_hca_workspace_size(const spattn_dims *dims) {
+    if (check_dims(dims) != SPATTN_OK) return 0;
+    return hca_workspace_bytes(dims);
+}
+
 spattn_status spattn_hca_attend(const spattn_dims *dims, const spattn_params *params, const void *q,
                                 const float *khat, const float *vhat, const int32_t *seq_lens, float *out,
-                                float *lse, spattn_stream_t stream) {
-    SP_TRY(check_dims(dims));
-    SP_TRY(check_params(params));
-    if (!q || !khat || !vhat || !seq_lens || !out || !lse)
-        return fail(SPATTN_ERR_INVALID_ARG, "q, khat, vhat, seq_lens, out, lse are required");
-    if (((uintptr_t)q | (uintptr_t)khat | (uintptr_t)vhat | (uintptr_t)out) & 15)
-        return fail(SPATTN_ERR_INVALID_ARG, "q, khat, vhat and out must be 16-byte aligned");
-    HcaAttendArgs a;
-    a.q = static_cast<const uint16_t *>(q);
-    a.khat = khat;
-    a.vhat = vhat;
-    a.seq_lens = seq_lens;
-    a.out = out;
-    a.lse = lse;
-    a.tq = dims->q_tokens;
-    a.hq = dims->num_q_heads;
-    a.hkv = dims->num_kv_heads;
-    a.max_blocks = dims->max_blocks_per_seq;
-    a.gmax = spattn_hca_entries(dims);
-    a.qscale = sm_scale_of(params) * kLog2e;
-    const int64_t rows = (int64_t)dims->batch * dims->q_tokens * dims->num_q_heads;
-    SP_TRY(cuda_ok(launch(hca_attend_kernel, dim3((unsigned)rows), dim3(32 * kHcaWarps), 0,
-                          reinterpret_cast<cudaStream_t>(stream), a),
-                   "hca_attend launch"));
-    return ok();
+                                float *lse, void *workspace, size_t workspace_bytes, spattn_stream_t stream) {
+    if (!lse) return fail(SPATTN_ERR_INVALID_ARG, "lse is required");
+    return launch_hca_attend(dims, params, q, khat, vhat, seq_lens, nullptr, nullptr, out, lse, workspace,
+                             workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+spattn_status spattn_hca_attend_merge(const spattn_dims *dims, const spattn_params *params, const void *q,
+                                      const float *khat, const float *vhat, const int32_t *seq_lens,
+                                      const float *out_other, const float *lse_other, float *out, float *lse,
+                                      void *workspace, size_t workspace_bytes, spattn_stream_t stream) {
+    if (!out_other || !lse_other) return fail(SPATTN_ERR_INVALID_ARG, "out_other and lse_other are required");
+    if ((uintptr_t)out_other & 15) return fail(SPATTN_ERR_INVALID_ARG, "out_other must be 16-byte aligned");
+    return launch_hca_attend(dims, params, q, khat, vhat, seq_lens, out_other, lse_other, out, lse, workspace,
+                             workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 spattn_status spattn_lse_merge(const spattn_dims *dims, const float *out_a, const float *lse_a,

@@ -11,7 +11,7 @@ uint8 e4m3fn codes) [num_pages][Hkv][64][128]; scales f32 [num_pages][Hkv];
 block_table int32 [B][max_blocks]; seq_lens int32 [B]; kbar f32
 [num_pages][Hkv][128]; scores f32 [B][Tq][Hkv][max_blocks]; sel_idx int32
 [B][Hkv][max_sel]; sel_count int32 [B][Hkv]; out f32 [B][Tq][Hq][128];
-lse f32 [B][Tq][Hq]; khat / vhat f32 [B][ceil(max_blocks / 2)][Hkv][128].
+lse f32 [B][Tq][Hq]; khat / vhat f32 [B][Hkv][ceil(max_blocks / 2)][128].
 """
 from __future__ import annotations
 
@@ -38,7 +38,8 @@ EXPORTS = ("spattn_required_max_sel", "spattn_compress_keys", "spattn_block_scor
            "spattn_select", "spattn_decode_workspace_size", "spattn_decode_selected",
            "spattn_decode", "spattn_last_error", "spattn_get_device_status", "spattn_version",
            "spattn_decode_selected_noalloc", "spattn_decode_selected_lse", "spattn_hca_entries",
-           "spattn_hca_pool", "spattn_hca_attend", "spattn_lse_merge")
+           "spattn_hca_pool", "spattn_hca_attend", "spattn_lse_merge", "spattn_hca_attend_merge",
+           "spattn_hca_workspace_size")
 
 
 class SpattnError(RuntimeError):
@@ -105,8 +106,10 @@ def load() -> ctypes.CDLL:
         "spattn_decode_selected_lse": ([P] * 14 + [ctypes.c_size_t, P], ctypes.c_int),
         "spattn_hca_entries": ([P], I32),
         "spattn_hca_pool": ([P] * 11, ctypes.c_int),
-        "spattn_hca_attend": ([P] * 9, ctypes.c_int),
+        "spattn_hca_attend": ([P] * 8 + [P, ctypes.c_size_t, P], ctypes.c_int),
+        "spattn_hca_workspace_size": ([P], ctypes.c_size_t),
         "spattn_lse_merge": ([P] * 8, ctypes.c_int),
+        "spattn_hca_attend_merge": ([P] * 10 + [P, ctypes.c_size_t, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -243,7 +246,7 @@ def hca_entries(block_table) -> int:
 
 def hca_pool(k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, khat, vhat, old_lens=None, *,
              q_tokens: int = 1, stream=None):
-    """Mean K and V of every 128-token entry: khat / vhat f32 [B][G][Hkv][128]."""
+    """Mean K and V of every 128-token entry: khat / vhat f32 [B][Hkv][G][128]."""
     num_pages, Hkv, P, D = k_cache.shape
     kv = KV_FP8_E4M3 if k_cache.dtype in (torch.uint8, torch.float8_e4m3fn) else KV_BF16
     dims = CDims(seq_lens.shape[0], q_tokens, Hkv, Hkv, D, P, num_pages, block_table.shape[1], 0, kv,
@@ -255,11 +258,31 @@ def hca_pool(k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, khat, vh
                                   _stream(stream)))
 
 
-def hca_attend(q, khat, vhat, seq_lens, out, lse, params: Params, *, k_cache, block_table, stream=None):
-    """Dense attention of every query row over its visible pooled entries."""
+def hca_workspace(q, k_cache, block_table) -> torch.Tensor:
+    """Workspace of hca_attend for these shapes (spattn_hca_workspace_size)."""
     dims = dims_for(q, k_cache, block_table)
-    _check(load().spattn_hca_attend(ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(khat), _p(vhat),
-                                    _p(seq_lens), _p(out), _p(lse), _stream(stream)))
+    n = load().spattn_hca_workspace_size(ctypes.byref(dims))
+    if n == 0:
+        raise SpattnError(1, "invalid dims")
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def hca_attend(q, khat, vhat, seq_lens, out, lse, params: Params, *, k_cache, block_table, workspace=None,
+               stream=None, merge_with=None):
+    """Dense attention of every query row over its visible pooled entries.
+    ``merge_with=(out_other, lse_other)``: the result merged with another
+    branch's (spattn_hca_attend_merge; lse may be None).  ``workspace``:
+    from hca_workspace(); allocated here when not given."""
+    dims = dims_for(q, k_cache, block_table)
+    ws = workspace if workspace is not None else hca_workspace(q, k_cache, block_table)
+    tail = [_p(ws), ws.numel() * ws.element_size(), _stream(stream)]
+    if merge_with is None:
+        _check(load().spattn_hca_attend(ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(khat),
+                                        _p(vhat), _p(seq_lens), _p(out), _p(lse), *tail))
+    else:
+        _check(load().spattn_hca_attend_merge(ctypes.byref(dims), ctypes.byref(params.c()), _p(q), _p(khat),
+                                              _p(vhat), _p(seq_lens), _p(merge_with[0]), _p(merge_with[1]),
+                                              _p(out), _p(lse), *tail))
 
 
 def lse_merge(out_a, lse_a, out_b, lse_b, out, lse=None, stream=None):

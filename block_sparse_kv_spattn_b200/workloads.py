@@ -97,6 +97,10 @@ WORKLOADS = {
     "decode_128k_b2": Workload("decode_128k_b2", batch=2, q_tokens=1, num_q_heads=32, num_kv_heads=8,
                                seq_len=131072, structure="zipf", mode="topp", top_p=0.9,
                                max_ratio=0.15, seed=1240),
+    # ... and with the HCA branch (profiling size of decode_128k_b8_hca)
+    "decode_128k_b2_hca": Workload("decode_128k_b2_hca", batch=2, q_tokens=1, num_q_heads=32, num_kv_heads=8,
+                                   seq_len=131072, structure="zipf", mode="topp", top_p=0.9,
+                                   max_ratio=0.15, hca=True, seed=1240),
     # 32 requests, lengths log-uniform in [8K, 256K], 64 q heads / 8 KV heads,
     # top-p 0.95 capped at 20 %.
     "ragged_b32": Workload("ragged_b32", batch=32, q_tokens=1, num_q_heads=64, num_kv_heads=8,

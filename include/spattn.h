@@ -310,7 +310,9 @@ spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params
  * (spattn_decode_selected_lse) through spattn_lse_merge, which is softmax
  * attention over the union of both key sets.
  *
- * khat / vhat are device fp32 [B][G][Hkv][d] with G = spattn_hca_entries().
+ * khat / vhat are device fp32 [B][Hkv][G][d] with G = spattn_hca_entries():
+ * the entries of one (request, KV head) are contiguous, so that the dense
+ * attention streams them in large copies.
  */
 #define SPATTN_HCA_BLOCKS 2
 
@@ -321,7 +323,7 @@ int32_t spattn_hca_entries(const spattn_dims *dims);
 /*
  * spattn_hca_pool -- mean K and V of each entry.
  *
- * khat[b][g][h][:] = mean over the tokens [128 g, min(L, 128 (g + 1))) of
+ * khat[b][h][g][:] = mean over the tokens [128 g, min(L, 128 (g + 1))) of
  * request b of K (dequantised with k_scale for fp8; fp32 sums), vhat the same
  * of V.  With old_lens == NULL every entry of every request is written
  * (entries past the end of a request: zeros); otherwise only the entries
@@ -335,19 +337,42 @@ spattn_status spattn_hca_pool(const spattn_dims *dims, const void *k_cache, cons
                               const int32_t *seq_lens, float *khat, float *vhat,
                               spattn_stream_t stream);
 
+/* Bytes of workspace spattn_hca_attend / spattn_hca_attend_merge need (the
+ * partial results of the shares of each request's entries).  Returns 0 on
+ * invalid dims. */
+size_t spattn_hca_workspace_size(const spattn_dims *dims);
+
 /*
  * spattn_hca_attend -- dense attention over the pooled entries.
  *
- * out[b][t][i][:] = softmax_g(sm_scale * q . khat[b][g][h]) vhat[b][g][h]
+ * out[b][t][i][:] = softmax_g(sm_scale * q . khat[b][h][g]) vhat[b][h][g]
  * over the visible entries g of (b, t), h = i / (Hq / Hkv); lse[b][t][i] =
  * ln of the softmax's denominator.  A row with no visible entry gets zeros
  * and -inf.  fp32 throughout; out and lse are device [B][Tq][Hq][d] and
- * [B][Tq][Hq] (both required).
+ * [B][Tq][Hq] (both required).  workspace: device, 256-byte aligned, at
+ * least spattn_hca_workspace_size() bytes (SPATTN_ERR_WORKSPACE otherwise);
+ * its contents need no initialisation.
  */
 spattn_status spattn_hca_attend(const spattn_dims *dims, const spattn_params *params,
                                 const void *q, const float *khat, const float *vhat,
                                 const int32_t *seq_lens, float *out, float *lse,
+                                void *workspace, size_t workspace_bytes,
                                 spattn_stream_t stream);
+
+/*
+ * spattn_hca_attend_merge -- spattn_hca_attend with the merge of
+ * spattn_lse_merge folded into its last kernel: out / lse = the softmax over
+ * the visible entries and another branch's keys together, given that
+ * branch's out_other ([B][Tq][Hq][d]) and lse_other ([B][Tq][Hq], as
+ * spattn_decode_selected_lse writes them).  lse may be NULL.  out and lse
+ * may be out_other and lse_other.  Workspace as spattn_hca_attend.
+ */
+spattn_status spattn_hca_attend_merge(const spattn_dims *dims, const spattn_params *params,
+                                      const void *q, const float *khat, const float *vhat,
+                                      const int32_t *seq_lens, const float *out_other,
+                                      const float *lse_other, float *out, float *lse,
+                                      void *workspace, size_t workspace_bytes,
+                                      spattn_stream_t stream);
 
 /*
  * spattn_lse_merge -- one softmax over two disjoint key sets from the two

@@ -125,7 +125,13 @@ def test_hca_entry_points_validate_on_the_host(lib):
                                None) == 1
     assert b"aligned" in lib.spattn_last_error()
     assert lib.spattn_hca_attend(ctypes.byref(d), ctypes.byref(p.c()), dummy, dummy, dummy, dummy, dummy,
-                                 None, None) == 1
+                                 None, dummy, 1 << 30, None) == 1
+    need = lib.spattn_hca_workspace_size(ctypes.byref(d))
+    assert need >= 2 * 8 * 16 * 4 * 128 * 4     # B * Hkv * max split * rows * d floats
+    assert lib.spattn_hca_attend(ctypes.byref(d), ctypes.byref(p.c()), dummy, dummy, dummy, dummy, dummy,
+                                 dummy, dummy, need - 1, None) == 4
+    assert lib.spattn_hca_attend_merge(ctypes.byref(d), ctypes.byref(p.c()), dummy, dummy, dummy, dummy, None,
+                                       dummy, dummy, None, dummy, need, None) == 1
     assert lib.spattn_lse_merge(ctypes.byref(d), dummy, dummy, dummy, None, dummy, None, None) == 1
     assert lib.spattn_lse_merge(ctypes.byref(_dims(head_dim=96)), dummy, dummy, dummy, dummy, dummy, None,
                                 None) == 2

@@ -20,7 +20,7 @@ import torch
 import oracle
 from block_sparse_kv_spattn_b200 import spattn
 from block_sparse_kv_spattn_b200.workloads import WORKLOADS, Workload, make_inputs
-from tests.cases import CHUNK2_TOPP, GQA8_TOPP, SMALL_FP8_CHUNK, SMALL_RAGGED, SMALL_TOPP
+from tests.cases import CHUNK2_TOPP, CHUNK16_FP8, GQA8_TOPP, MQA16_TOPK, SMALL_FP8_CHUNK, SMALL_RAGGED, SMALL_TOPP
 from tests.oracle_io import dims_of, host_arrays, params_of
 from tests.parity import OUT_TOL, lib_params, run_library
 
@@ -39,7 +39,7 @@ def _lib(cuda):
 def gpu_pool(inp):
     kc, bt = inp["k_cache"], inp["block_table"]
     G = spattn.hca_entries(bt)
-    shape = (bt.shape[0], G, kc.shape[1], kc.shape[3])
+    shape = (bt.shape[0], kc.shape[1], G, kc.shape[3])    # [B][Hkv][G][d]
     khat = torch.full(shape, float("nan"), device="cuda")
     vhat = torch.full(shape, float("nan"), device="cuda")
     spattn.hca_pool(kc, inp["v_cache"], inp["k_scale"], inp["v_scale"], bt, inp["seq_lens"], khat, vhat)
@@ -61,6 +61,11 @@ def oracle_pool(inp):
                            a["block_table"], a["seq_lens"], GROUP)
 
 
+def host(t):
+    """GPU entries [B][Hkv][G][d] -> the oracle's [B][G][Hkv][d], float64."""
+    return t.permute(0, 2, 1, 3).double().cpu().numpy()
+
+
 def _max_err(gpu, ref):
     g = gpu.double().cpu().numpy() if torch.is_tensor(gpu) else gpu
     both_inf = np.isinf(g) & np.isinf(ref) & (np.sign(g) == np.sign(ref))
@@ -69,7 +74,7 @@ def _max_err(gpu, ref):
     return float(np.nan_to_num(d, nan=np.inf).max()) if d.size else 0.0
 
 
-HCA_CASES = [SMALL_TOPP, SMALL_FP8_CHUNK, SMALL_RAGGED, GQA8_TOPP, CHUNK2_TOPP]
+HCA_CASES = [SMALL_TOPP, SMALL_FP8_CHUNK, SMALL_RAGGED, GQA8_TOPP, CHUNK2_TOPP, MQA16_TOPK, CHUNK16_FP8]
 
 
 @pytest.mark.parametrize("w", HCA_CASES, ids=lambda w: w.name)
@@ -79,7 +84,7 @@ def test_hca_pool_parity(w):
     assert spattn.device_status() == 0
     rk, rv = oracle_pool(inp)
     for g, r in ((khat, rk), (vhat, rv)):
-        err = np.abs(g.double().cpu().numpy() - r) / (1.0 + np.abs(r))
+        err = np.abs(host(g) - r) / (1.0 + np.abs(r))
         assert err.max() <= POOL_TOL
 
 
@@ -90,8 +95,8 @@ def test_hca_attend_parity(w):
     out, lse = gpu_hca_attend(inp, khat, vhat)
     assert spattn.device_status() == 0
     a = host_arrays(inp)
-    ro, rl = oracle.hca_attend(dims_of(inp), params_of(w), a["q"], khat.double().cpu().numpy(),
-                               vhat.double().cpu().numpy(), a["seq_lens"], GROUP)
+    ro, rl = oracle.hca_attend(dims_of(inp), params_of(w), a["q"], host(khat),
+                               host(vhat), a["seq_lens"], GROUP)
     assert _max_err(out, ro) <= HCA_TOL
     assert _max_err(lse, rl) <= HCA_TOL * (1 + np.abs(np.nan_to_num(rl, neginf=0)).max())
     assert torch.equal(torch.isinf(lse).cpu(), torch.from_numpy(np.isinf(rl)))
@@ -169,6 +174,32 @@ def hybrid_gpu(inp):
     return gpu, khat, vhat, out, lse
 
 
+def test_hca_attend_merge_is_attend_then_lse_merge():
+    """spattn_hca_attend_merge against the oracle's merge of the oracle's
+    two branches (GPU selection and entries as inputs), and against the
+    GPU's own two-launch composition."""
+    for w in (SMALL_TOPP, CHUNK2_TOPP, GQA8_TOPP):
+        inp = make_inputs(w, device="cuda")
+        gpu, khat, vhat, out2, lse2 = hybrid_gpu(inp)
+        params = lib_params(w)
+        dims = spattn.dims_for(inp["q"], inp["k_cache"], inp["block_table"], gpu["max_sel"])
+        ws = spattn.alloc_workspace(dims, params, "cuda")
+        o_s = torch.empty_like(gpu["out"])
+        l_s = torch.empty(tuple(inp["q"].shape[:3]), device="cuda")
+        spattn.decode_selected(inp["q"], inp["k_cache"], inp["v_cache"], inp["k_scale"], inp["v_scale"],
+                               inp["block_table"], inp["seq_lens"], gpu["sel_idx"], gpu["sel_count"], o_s, ws,
+                               params, lse=l_s)
+        out = torch.full_like(o_s, float("nan"))
+        lse = torch.full_like(l_s, float("nan"))
+        spattn.hca_attend(inp["q"], khat, vhat, inp["seq_lens"], out, lse, params, k_cache=inp["k_cache"],
+                          block_table=inp["block_table"], merge_with=(o_s, l_s))
+        assert spattn.device_status() == 0
+        ro, rl = hybrid_oracle(inp, gpu, khat, vhat)
+        assert _max_err(out, ro) <= OUT_TOL[w.kv_fp8]
+        assert _max_err(lse, rl) <= LSE_TOL
+        assert _max_err(out, out2.double().cpu().numpy()) <= 1e-5
+
+
 def hybrid_oracle(inp, gpu, khat, vhat, requests=None):
     """The oracle's sparse branch over the GPU's selection and its HCA branch
     over the GPU's pooled entries, merged by the oracle."""
@@ -179,7 +210,7 @@ def hybrid_oracle(inp, gpu, khat, vhat, requests=None):
     o_s, l_s = oracle.attend(dims, prm, a["q"], a["k_cache"], a["v_cache"], a["k_scale"], a["v_scale"],
                              a["block_table"], a["seq_lens"], gpu["sel_idx"].cpu().numpy(),
                              gpu["sel_count"].cpu().numpy(), units=units, with_lse=True)
-    o_h, l_h = oracle.hca_attend(dims, prm, a["q"], khat.double().cpu().numpy(), vhat.double().cpu().numpy(),
+    o_h, l_h = oracle.hca_attend(dims, prm, a["q"], host(khat), host(vhat),
                                  a["seq_lens"], GROUP)
     return oracle.lse_merge(o_s, l_s, o_h, l_h)
 
@@ -200,8 +231,8 @@ def test_hybrid_full_size_sampled():
     inp = make_inputs(w, device="cuda")
     gpu, khat, vhat, out, lse = hybrid_gpu(inp)
     rk, rv = oracle_pool(inp)
-    assert (np.abs(khat.double().cpu().numpy() - rk) / (1 + np.abs(rk))).max() <= POOL_TOL
-    assert (np.abs(vhat.double().cpu().numpy() - rv) / (1 + np.abs(rv))).max() <= POOL_TOL
+    assert (np.abs(host(khat) - rk) / (1 + np.abs(rk))).max() <= POOL_TOL
+    assert (np.abs(host(vhat) - rv) / (1 + np.abs(rv))).max() <= POOL_TOL
     reqs = [0, 7]
     ro, rl = hybrid_oracle(inp, gpu, khat, vhat, requests=reqs)
     assert _max_err(out[reqs], ro[reqs]) <= OUT_TOL[False]
@@ -220,10 +251,10 @@ def test_hca_edge_lengths():
     out, lse = gpu_hca_attend(inp, khat, vhat)
     assert spattn.device_status() == 0
     rk, rv = oracle_pool(inp)
-    assert (np.abs(khat.double().cpu().numpy() - rk) / (1 + np.abs(rk))).max() <= POOL_TOL
+    assert (np.abs(host(khat) - rk) / (1 + np.abs(rk))).max() <= POOL_TOL
     a = host_arrays(inp)
-    ro, rl = oracle.hca_attend(dims_of(inp), params_of(w), a["q"], khat.double().cpu().numpy(),
-                               vhat.double().cpu().numpy(), a["seq_lens"], GROUP)
+    ro, rl = oracle.hca_attend(dims_of(inp), params_of(w), a["q"], host(khat),
+                               host(vhat), a["seq_lens"], GROUP)
     assert _max_err(out, ro) <= HCA_TOL
     assert torch.equal(torch.isinf(lse).cpu(), torch.from_numpy(np.isinf(rl)))
     # request 0 sees nothing; request 1 (one token): only its last query
@@ -243,7 +274,7 @@ def test_incremental_pool_matches_full():
     old = torch.tensor([64 * 20 + 10], dtype=torch.int32, device="cuda")
     new = old + 60
     G = spattn.hca_entries(bt)
-    shape = (1, G, kc.shape[1], 128)
+    shape = (1, kc.shape[1], G, 128)
     inc = torch.zeros(shape, device="cuda")
     inc_v = torch.zeros(shape, device="cuda")
     spattn.hca_pool(kc, vc, inp["k_scale"], inp["v_scale"], bt, old, inc, inc_v)
