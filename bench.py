@@ -7,10 +7,13 @@ One step is one pass of the whole decode path over the workload's batch:
 incremental key compression of each request's tail block (on a forked
 graph branch: the tail block is local, never scored), block scores,
 selection (sink + local + top-p/top-k), sparse attention and the split
-merge, all through the C ABI (captured once into CUDA graphs and replayed).
-Inputs are seeded synthetic data resident in HBM; L2 is flushed (a 512 MB
-write, then a 512 MB read that writes the flush's dirty lines back) between
-timed steps, outside the timed events.
+merge (and, for the HCA workloads, the dense branch over pooled 128-token
+entries merged with the sparse one), all through the C ABI, captured once
+into one CUDA graph per step and replayed.  Event-record nodes inside the
+graph time the step and its parts on the device.  Inputs are seeded
+synthetic data resident in HBM; L2 is flushed (a 512 MB write, then a 512 MB
+read that writes the flush's dirty lines back) before every timed step,
+outside the timed events.
 
 Metric: selected-KV HBM GB/s = algorithmic bytes of a step (kept K+V tiles,
 fp8 scales, compressed keys of the scored middle blocks, q, out) / step time,
@@ -271,21 +274,22 @@ def run_native(args, rank, world, local_rank):
     status = spattn.device_status()
     if status:
         raise RuntimeError(f"device status {status:#x}")
+    # the whole step in one graph; events recorded as graph nodes time its
+    # parts on the device (start, after the front, after the sparse
+    # attention, after the HCA branch)
+    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        g_front, g_attn, g_hca = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_front, stream=s):
+        g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step, stream=s):
+            marks[0].record()
             front()
-        with torch.cuda.graph(g_attn, stream=s):
+            marks[1].record()
             attend()
-        if w.hca:
-            with torch.cuda.graph(g_hca, stream=s):
-                hca()
-
-    def hca_replay():
-        if w.hca:
-            g_hca.replay()
+            marks[2].record()
+            hca()
+            marks[3].record()
     torch.cuda.current_stream().wait_stream(s)
     launches_per_step = 5          # compress, scores, select, attention, merge
     if w.hca:
@@ -293,12 +297,10 @@ def run_native(args, rank, world, local_rank):
 
     for _ in range(args.warmup):
         flush_l2()
-        g_front.replay()
-        g_attn.replay()
-        hca_replay()
+        g_step.replay()
     torch.cuda.synchronize()
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    step_ms, attn_ms, hca_list = [], [], []
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -307,25 +309,19 @@ def run_native(args, rank, world, local_rank):
               if hasattr(props, "pci_bus_id") else str(local_rank))
     with Clocks(smi_id) as clk:
         t_wall = time.perf_counter()
-        # hold the stream for ~50 ms so the host queues steps ahead of the
-        # device: the events then time device work, not host submission
-        torch.cuda._sleep(int(0.05 * props.clock_rate * 1e3))
         for i in range(K):
             flush_l2()
-            ev[i][0].record()
-            g_front.replay()
-            ev[i][1].record()
-            g_attn.replay()
-            ev[i][2].record()
-            hca_replay()
-            ev[i][3].record()
+            g_step.replay()
+            marks[3].synchronize()
+            step_ms.append(marks[0].elapsed_time(marks[3]))
+            attn_ms.append(marks[1].elapsed_time(marks[2]))
+            hca_list.append(marks[2].elapsed_time(marks[3]))
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     if world > 1:
         torch.distributed.barrier()
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    hca_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / K
+    hca_ms = sum(hca_list) / K
+    front_ms = sum(st - at - hc for st, at, hc in zip(step_ms, attn_ms, hca_list)) / K
     total_ms = sum(step_ms)
     bts = step_bytes(inp, sel_count)
     status = spattn.device_status()
@@ -342,9 +338,7 @@ def run_native(args, rank, world, local_rank):
         e2e_ev[i][0].record()
         q.copy_(q_h, non_blocking=True)
         sl.copy_(sl_h, non_blocking=True)
-        g_front.replay()
-        g_attn.replay()
-        hca_replay()
+        g_step.replay()
         out_h.copy_(out, non_blocking=True)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
@@ -389,6 +383,7 @@ def run_native(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": q.numel() * 2 + sl.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 4},
+        "front_ms": round(front_ms, 5),
         "gpu_launches": K * launches_per_step,
         "clocks": clk.summary(),
         "wall_s": round(t_wall, 3),

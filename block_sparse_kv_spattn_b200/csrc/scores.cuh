@@ -72,6 +72,9 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     const int j0 = blockIdx.x * a.bpc;
     const int G = a.hq / HKV;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the selection grid that follows may be scheduled now: it waits for
+    // this grid's completion before it reads the scores
+    asm volatile("griddepcontrol.launch_dependents;");
 
     int L = a.seq_lens[b];
     if (L < 0 || L > a.max_blocks * kBlock) {

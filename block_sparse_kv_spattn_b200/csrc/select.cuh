@@ -322,13 +322,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     }
     const int bh = blockIdx.x;
     const int b = bh / a.hkv, h = bh % a.hkv;
-    // the first token's score row into L1 while the length is fetched
+    // launched early (programmatic dependent launch): wait for the previous
+    // grid in the stream (the scoring) to complete before reading anything
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    int L = a.seq_lens[b];
+    // the first token's score row into L1
     {
         const float *row0 = a.scores + ((int64_t)b * a.tq * a.hkv + h) * a.max_blocks;
         for (int i = threadIdx.x * 32; i < a.n_mid_cap + a.sink; i += blockDim.x * 32)
             asm volatile("prefetch.global.L1 [%0];" ::"l"(row0 + i));
     }
-    int L = a.seq_lens[b];
     if (L < 0 || L > a.max_blocks * kBlock) {
         if (threadIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
         L = 0;

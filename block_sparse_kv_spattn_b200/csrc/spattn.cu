@@ -217,9 +217,8 @@ DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
 
 // ------------------------------------------------------------- launches
 
-// Plain stream-ordered launch through cudaLaunchKernelEx.  (Programmatic
-// dependent launch was measured on this path and lost: an early-scheduled
-// successor takes SM resources the predecessor's tail still uses.)
+// Plain stream-ordered launch through cudaLaunchKernelEx.  (The split merge
+// after the attention kernel launched early was measured slower.)
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args &&...args) {
@@ -230,6 +229,26 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     cfg.stream = st;
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Launch whose CTAs may be scheduled before the previous kernel in the
+// stream has finished (programmatic dependent launch): the kernel runs its
+// input-independent prologue, then waits (griddepcontrol.wait) for the
+// previous grid's completion and memory before reading its results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_early(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         Args &&...args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -318,7 +337,7 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
     // passes (measured: 512 beat 1024 by 15-25 % on 2K-4K middle blocks)
     const int nm = n_mid_cap(d, p);
     const int threads = nm <= 1024 ? 256 : (nm <= 4096 ? 512 : kSelThreads);
-    return cuda_ok(launch(select_kernel, dim3(d->batch * d->num_kv_heads), dim3(threads), smem, st, a),
+    return cuda_ok(launch_early(select_kernel, dim3(d->batch * d->num_kv_heads), dim3(threads), smem, st, a),
                    "select launch");
 }
 
