@@ -224,7 +224,7 @@ def run_native(args, rank, world, local_rank):
     # compressed keys are never scored (local blocks are always kept), so the
     # append-side compression runs on a forked branch beside scoring.
     assert Tq <= (w.local_blocks - 1) * w.block_size + 1, "append would touch a middle block"
-    side = torch.cuda.Stream()
+    side, side2 = torch.cuda.Stream(), torch.cuda.Stream()
 
     anchored = w.mode == "topp_anchor"   # the local blocks are scored: compress first
 
@@ -248,12 +248,16 @@ def run_native(args, rank, world, local_rank):
             with torch.cuda.stream(side):
                 spattn.compress_keys(kc, ks, bt, sl, kbar, old_lens=old_lens, num_q_heads=w.num_q_heads,
                                      q_tokens=Tq)
-                if w.hca:
-                    spattn.hca_pool(kc, vc, ks, vs, bt, sl, khat, vhat, old_lens=old_lens, q_tokens=Tq)
+        if w.hca:   # the appended tokens' pooled entries, on a branch of their own
+            side2.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side2):
+                spattn.hca_pool(kc, vc, ks, vs, bt, sl, khat, vhat, old_lens=old_lens, q_tokens=Tq)
         spattn.block_scores(q, kbar, bt, sl, scores, params, k_cache=kc)
         spattn.select(scores, sl, sel_idx, sel_count, params, q=q, k_cache=kc, block_table=bt)
         if not anchored:
             torch.cuda.current_stream().wait_stream(side)
+        if w.hca:
+            torch.cuda.current_stream().wait_stream(side2)
 
     def attend():  # sparse attention + split merge
         if not w.hca:

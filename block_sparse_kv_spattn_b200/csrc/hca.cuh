@@ -26,15 +26,22 @@ struct HcaPoolArgs {
     int hkv, num_pages, max_blocks, gmax;
 };
 
-// Grid (gx, B), Hkv warps: warp h sums K and V of KV head h over an entry's
-// tokens (lane: 4 columns) in fp32, then divides by the token count; the
-// CTAs stride over the entries.  Without old_lens every entry is written
-// (zeros past the end of the request); with old_lens only the entries that
-// hold a token of [old_len, L).
+constexpr int kHcaPoolThreads = 512;
+
+// Grid (gx, B), kHcaPoolThreads threads; the CTAs stride over the entries.
+// Without old_lens every entry is written (zeros past the end of the
+// request); with old_lens only the entries that hold a token of
+// [old_len, L).  Per entry, half-warp j of 32 takes KV head j % Hkv and every
+// (32 / Hkv)-th token from token j / Hkv, 8 columns per lane in fp32 (fp8
+// codes times their page's scale); the half-warps' sums are combined in a
+// fixed order through shared memory and divided by the token count.
 template <bool FP8>
-__global__ void __launch_bounds__(16 * 32) hca_pool_kernel(HcaPoolArgs a) {
-    const int b = blockIdx.y, h = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (h >= a.hkv) return;
+__global__ void __launch_bounds__(kHcaPoolThreads) hca_pool_kernel(HcaPoolArgs a) {
+    __shared__ float4 s_k[32][32], s_v[32][32];   // [half-warp][16 lanes x 8 columns as 2 float4]
+    __shared__ int s_page[kHcaGroupBlocks];
+    const int b = blockIdx.y;
+    const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
+    const int h = hw % a.hkv, tl = hw / a.hkv, ntl = 32 / a.hkv;
     const int L = a.seq_lens[b];
     if (L < 0 || L > a.max_blocks * kBlock) {
         if (threadIdx.x == 0 && blockIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
@@ -47,50 +54,66 @@ __global__ void __launch_bounds__(16 * 32) hca_pool_kernel(HcaPoolArgs a) {
     }
     for (int g = g_lo + blockIdx.x; g < g_hi; g += gridDim.x) {
         const int t0 = g * kHcaTokens, t1 = min(L, t0 + kHcaTokens);
-        float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
-        for (int blk = 0; blk < kHcaGroupBlocks && t0 + blk * kBlock < t1; ++blk) {
-            const int j = g * kHcaGroupBlocks + blk;
-            const int page = a.block_table[(int64_t)b * a.max_blocks + j];
-            if (page < 0 || page >= a.num_pages) {
-                if (lane == 0) flag(SPATTN_DEV_BAD_PAGE);
-                continue;
-            }
-            const int n = min(kBlock, t1 - j * kBlock);
-            const int64_t base = ((int64_t)page * a.hkv + h) * kBlock * kHeadDim + lane * 4;
-            float ksc = 1.f, vsc = 1.f;
-            if (FP8) {
-                ksc = a.k_scale[(int64_t)page * a.hkv + h];
-                vsc = a.v_scale[(int64_t)page * a.hkv + h];
-            }
-            float4 bk = make_float4(0.f, 0.f, 0.f, 0.f), bv = bk;
-#pragma unroll 4
-            for (int t = 0; t < n; ++t) {
-                float kx[4], vx[4];
-                if (FP8) {
-                    const uint32_t ku = *reinterpret_cast<const uint32_t *>(a.k_cache + base + t * kHeadDim);
-                    const uint32_t vu = *reinterpret_cast<const uint32_t *>(a.v_cache + base + t * kHeadDim);
-                    e4m3x2_to_f32((uint16_t)(ku & 0xffffu), kx[0], kx[1]);
-                    e4m3x2_to_f32((uint16_t)(ku >> 16), kx[2], kx[3]);
-                    e4m3x2_to_f32((uint16_t)(vu & 0xffffu), vx[0], vx[1]);
-                    e4m3x2_to_f32((uint16_t)(vu >> 16), vx[2], vx[3]);
-                } else {
-                    const uint2 ku = *reinterpret_cast<const uint2 *>(a.k_cache + (base + t * kHeadDim) * 2);
-                    const uint2 vu = *reinterpret_cast<const uint2 *>(a.v_cache + (base + t * kHeadDim) * 2);
-                    kx[0] = bf16lo(ku.x), kx[1] = bf16hi(ku.x), kx[2] = bf16lo(ku.y), kx[3] = bf16hi(ku.y);
-                    vx[0] = bf16lo(vu.x), vx[1] = bf16hi(vu.x), vx[2] = bf16lo(vu.y), vx[3] = bf16hi(vu.y);
+        if (threadIdx.x < kHcaGroupBlocks) {
+            const int j = g * kHcaGroupBlocks + threadIdx.x;
+            int page = -1;
+            if (t0 + (int)threadIdx.x * kBlock < t1) {
+                page = a.block_table[(int64_t)b * a.max_blocks + j];
+                if (page < 0 || page >= a.num_pages) {
+                    flag(SPATTN_DEV_BAD_PAGE);
+                    page = -1;
                 }
-                bk.x += kx[0], bk.y += kx[1], bk.z += kx[2], bk.w += kx[3];
-                bv.x += vx[0], bv.y += vx[1], bv.z += vx[2], bv.w += vx[3];
             }
-            sk.x = fmaf(bk.x, ksc, sk.x), sk.y = fmaf(bk.y, ksc, sk.y);
-            sk.z = fmaf(bk.z, ksc, sk.z), sk.w = fmaf(bk.w, ksc, sk.w);
-            sv.x = fmaf(bv.x, vsc, sv.x), sv.y = fmaf(bv.y, vsc, sv.y);
-            sv.z = fmaf(bv.z, vsc, sv.z), sv.w = fmaf(bv.w, vsc, sv.w);
+            s_page[threadIdx.x] = page;
         }
+        __syncthreads();
+        float k8[8], v8[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) k8[c] = v8[c] = 0.f;
+#pragma unroll 4
+        for (int t = t0 + tl; t < t1; t += ntl) {
+            const int page = s_page[(t - t0) / kBlock];
+            if (page < 0) continue;
+            const int64_t off = (((int64_t)page * a.hkv + h) * kBlock + (t % kBlock)) * kHeadDim + hl * 8;
+            float kx[8], vx[8];
+            if (FP8) {
+                const float ks = a.k_scale[(int64_t)page * a.hkv + h], vs = a.v_scale[(int64_t)page * a.hkv + h];
+                e4m3x8_to_f32(*reinterpret_cast<const uint2 *>(a.k_cache + off), kx);
+                e4m3x8_to_f32(*reinterpret_cast<const uint2 *>(a.v_cache + off), vx);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    k8[c] = fmaf(kx[c], ks, k8[c]);
+                    v8[c] = fmaf(vx[c], vs, v8[c]);
+                }
+            } else {
+                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(a.k_cache + off * 2), kx);
+                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(a.v_cache + off * 2), vx);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    k8[c] += kx[c];
+                    v8[c] += vx[c];
+                }
+            }
+        }
+        s_k[hw][2 * hl] = make_float4(k8[0], k8[1], k8[2], k8[3]);
+        s_k[hw][2 * hl + 1] = make_float4(k8[4], k8[5], k8[6], k8[7]);
+        s_v[hw][2 * hl] = make_float4(v8[0], v8[1], v8[2], v8[3]);
+        s_v[hw][2 * hl + 1] = make_float4(v8[4], v8[5], v8[6], v8[7]);
+        __syncthreads();
+        // thread -> (K or V, head, 4 columns): sum the head's half-warps in order
         const float inv = t1 > t0 ? 1.f / (float)(t1 - t0) : 0.f;
-        const int64_t o = (((int64_t)b * a.hkv + h) * a.gmax + g) * kHeadDim + lane * 4;
-        *reinterpret_cast<float4 *>(a.khat + o) = make_float4(sk.x * inv, sk.y * inv, sk.z * inv, sk.w * inv);
-        *reinterpret_cast<float4 *>(a.vhat + o) = make_float4(sv.x * inv, sv.y * inv, sv.z * inv, sv.w * inv);
+        for (int task = threadIdx.x; task < 2 * a.hkv * 32; task += kHcaPoolThreads) {
+            const int kv = task / (a.hkv * 32), hh = (task / 32) % a.hkv, c4 = task % 32;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < ntl; ++j) {
+                const float4 x = kv ? s_v[j * a.hkv + hh][c4] : s_k[j * a.hkv + hh][c4];
+                acc.x += x.x, acc.y += x.y, acc.z += x.z, acc.w += x.w;
+            }
+            float *dst = kv ? a.vhat : a.khat;
+            reinterpret_cast<float4 *>(dst + (((int64_t)b * a.hkv + hh) * a.gmax + g) * kHeadDim)[c4] =
+                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        }
+        __syncthreads();   // s_page and the partials are reused by the next entry
     }
 }
 

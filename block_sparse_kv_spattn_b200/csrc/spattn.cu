@@ -842,7 +842,7 @@ spattn_status spattn_hca_pool(const spattn_dims *dims, const void *k_cache, cons
     // incremental: the entries of the appended tokens (q_tokens of them, the
     // CTAs stride over more if a request grew further)
     const int gx = old_lens ? (dims->q_tokens + kHcaTokens - 1) / kHcaTokens + 1 : a.gmax;
-    const dim3 grid(gx, dims->batch), block(32 * dims->num_kv_heads);
+    const dim3 grid(gx, dims->batch), block(kHcaPoolThreads);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (fp8)
         hca_pool_kernel<true><<<grid, block, 0, st>>>(a);
