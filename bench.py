@@ -48,7 +48,7 @@ from block_sparse_kv_spattn_b200.workloads import BENCH_WORKLOAD, WORKLOADS, mak
 METRIC = "selected-KV HBM GB/s (% of ~8 TB/s) and decode queries/s at 128K ctx, 1 B200"
 FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
-ATTN_SOURCES = ["common.cuh", "attention.cuh", "tcgen05.cuh", "attention_tc.cuh"]
+ATTN_SOURCES = ["common.cuh", "attention.cuh", "tcgen05.cuh", "attention_tc.cuh", "attention_tcw.cuh"]
 
 
 def _peaks():
@@ -74,7 +74,8 @@ def attn_label(w) -> str:
     if not w.kv_fp8 and rows <= 16:
         rq = 4 if rows <= 4 else (8 if rows <= 8 else 16)
         return f"attention (attn_tc_kernel<{rq}> on tcgen05 + merge_kernel, one decode_selected call)"
-    return "attention (attn_kernel + merge_kernel, one decode_selected call)"
+    return (f"attention (attn_tcw_kernel<{'fp8' if w.kv_fp8 else 'bf16'}> on tcgen05, query rows on M, "
+            f"+ merge_kernel, one decode_selected call)")
 
 
 def measured_traffic(units_in_launch: float):

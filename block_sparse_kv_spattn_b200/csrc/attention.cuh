@@ -517,7 +517,8 @@ struct MergeArgs {
     float *out;                 // [B][Tq][Hq][D]
     float *lse;                 // nullable: [B][Tq][Hq], ln of the row's sum of exp(logit)
     int batch, tq, hq, hkv, group, rows, units, max_sel, ctas;
-    int wslots;                 // partial records per (CTA, unit): 1, or one per tensor-core softmax warp
+    int wslots;                 // partial records per (CTA, unit): 1, 2 (hi / lo parts) or 4 (per softmax warp)
+    int pairs;                  // 4 records: warp w's pair w / 2 took only tiles of its parity
 };
 
 constexpr int kMergeMaxWarps = 8;   // warps per output row, for units split over many CTAs
@@ -534,7 +535,7 @@ __device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int x, int c
     const int64_t ia = (pre > lo_c ? pre : lo_c) - lo_c;
     const int64_t ib = (pre + cnt < hi_c ? pre + cnt : hi_c) - lo_c;
     if (ib <= ia) return -1;
-    if (a.wslots > 1 && ib - ia < 2 && (ia & 1) != (w >> 1)) return -1;
+    if (a.pairs && ib - ia < 2 && (ia & 1) != (w >> 1)) return -1;
     return ((int64_t)cc + unit) * a.wslots + w;
 }
 

@@ -21,6 +21,7 @@
 #include "select.cuh"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "attention_tcw.cuh"
 #include "hca.cuh"
 
 using namespace spattn;
@@ -140,9 +141,14 @@ float sm_scale_of(const spattn_params *p) {
 
 int rows_of(const spattn_dims *d) { return d->q_tokens * (d->num_q_heads / d->num_kv_heads); }
 
-// Attention runs on the tensor cores for bf16 caches with at most kTcNQ
-// query rows per KV head, on CUDA cores otherwise.
+// Attention runs on the tensor cores: attn_tc_kernel for bf16 caches with
+// at most kTcNQ query rows per KV head, attn_tcw_kernel for the rest (fp8
+// caches, or up to kTcwRows rows).
 bool uses_tc(const spattn_dims *d) { return d->kv_dtype == SPATTN_KV_BF16 && rows_of(d) <= kTcNQ; }
+
+// Partial records per (CTA, unit) slot: one per softmax warp (attn_tc), one
+// (attn_tcw).
+int records_per_slot(const spattn_dims *d) { return uses_tc(d) ? kTcWarpSlots : 1; }
 
 int rg_of(int rows) {
     const int rg = (rows + 3) / 4;
@@ -194,12 +200,11 @@ struct DecodeLayout {
 };
 
 // Workspace: [scores] | partial outputs | partial (max, sum).  (C_max +
-// units) slots of `rows` query rows, one partial record per slot (CUDA-core
-// kernel) or one per softmax warp (tensor-core kernel, kTcWarpSlots).
+// units) slots of `rows` query rows, records_per_slot() records per slot.
 DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
     DecodeLayout L{};
     const int64_t units = (int64_t)d->batch * d->num_kv_heads;
-    const int64_t slots = (kMaxAttnCtas + units) * (uses_tc(d) ? kTcWarpSlots : 1);
+    const int64_t slots = (kMaxAttnCtas + units) * records_per_slot(d);
     const int64_t rows = rows_of(d);
     size_t off = 0;
     L.scores_off = 0;
@@ -381,19 +386,22 @@ EncodeTiledFn g_encode = nullptr;
 
 // 2-D view of a bf16 cache as [num_pages * Hkv * 64 token rows][128], boxes
 // of 64 x 64 with 128-byte swizzle (the tensor-core operand layout).
-spattn_status kv_tensor_map(CUtensorMap *m, const void *base, int64_t rows) {
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_encode) {
-            void *fn = nullptr;
-            cudaDriverEntryPointQueryResult q;
-            SP_TRY(cuda_ok(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q),
-                           "cudaGetDriverEntryPoint"));
-            if (!fn || q != cudaDriverEntryPointSuccess)
-                return fail(SPATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-        }
+spattn_status kv_tensor_map_encoder() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        SP_TRY(cuda_ok(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q),
+                       "cudaGetDriverEntryPoint"));
+        if (!fn || q != cudaDriverEntryPointSuccess)
+            return fail(SPATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
+    return SPATTN_OK;
+}
+
+spattn_status kv_tensor_map(CUtensorMap *m, const void *base, int64_t rows) {
+    SP_TRY(kv_tensor_map_encoder());
     const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
     const cuuint32_t box[2] = {64, 64};
@@ -403,6 +411,43 @@ spattn_status kv_tensor_map(CUtensorMap *m, const void *base, int64_t rows) {
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(SPATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return SPATTN_OK;
+}
+
+// 2-D view of an fp8 cache as [num_pages * Hkv * 64 token rows][128 bytes],
+// boxes of one whole (page, head) tile (64 rows x 128 bytes), 128-byte
+// swizzle (the staging buffer the converter warps read).
+spattn_status kv_tensor_map_u8(CUtensorMap *m, const void *base, int64_t rows) {
+    SP_TRY(kv_tensor_map_encoder());
+    const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim};
+    const cuuint32_t box[2] = {128, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SPATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SPATTN_OK;
+}
+
+// Tensor-core path for many rows and fp8 caches: one CTA per SM.
+template <bool FP8>
+spattn_status launch_attn_tcw(AttnArgs &a, const void *k_cache, const void *v_cache, int sms, cudaStream_t st,
+                              int *ctas_out) {
+    CUtensorMap kmap, vmap;
+    const int64_t rows = (int64_t)a.num_pages * a.hkv * kBlock;
+    if (FP8) {
+        SP_TRY(kv_tensor_map_u8(&kmap, k_cache, rows));
+        SP_TRY(kv_tensor_map_u8(&vmap, v_cache, rows));
+    } else {
+        SP_TRY(kv_tensor_map(&kmap, k_cache, rows));
+        SP_TRY(kv_tensor_map(&vmap, v_cache, rows));
+    }
+    const int smem = TcwLayout<FP8>::kSmem;
+    SP_TRY(ensure_smem((const void *)attn_tcw_kernel<FP8>, smem));
+    const int ctas = std::min(kMaxAttnCtas, sms);
+    *ctas_out = ctas;
+    return cuda_ok(launch(attn_tcw_kernel<FP8>, dim3(ctas), dim3(kTcwThreads), smem, st, kmap, vmap, a),
+                   "attention (tensor core, many rows) launch");
 }
 
 // Tensor-core path: bf16 caches, at most kTcNQ query rows per KV head.  One
@@ -479,7 +524,8 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     if (tc)
         SP_TRY(launch_attn_tc(a, k_cache, v_cache, sms, st, &ctas));
     else
-        SP_TRY(fp8 ? launch_attn_rg<true>(rg, a, sms, st, &ctas) : launch_attn_rg<false>(rg, a, sms, st, &ctas));
+        SP_TRY(fp8 ? launch_attn_tcw<true>(a, k_cache, v_cache, sms, st, &ctas)
+                   : launch_attn_tcw<false>(a, k_cache, v_cache, sms, st, &ctas));
 
     MergeArgs m;
     m.part_o = a.part_o;
@@ -496,7 +542,8 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.units = a.units;
     m.max_sel = d->max_sel;
     m.ctas = ctas;
-    m.wslots = tc ? kTcWarpSlots : 1;
+    m.wslots = records_per_slot(d);
+    m.pairs = tc ? 1 : 0;
     // one CTA per output row; warps for the records a unit gets on average
     // (CTAs per unit + 1, times the records per CTA), 32 per warp
     const int64_t nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
@@ -560,6 +607,13 @@ constexpr bool tc_layout_ok() {
 }
 static_assert(tc_layout_ok<4>() && tc_layout_ok<8>() && tc_layout_ok<16>(),
               "one CTA per SM; even stage count; swizzled operand tiles on 1024-byte boundaries");
+template <bool FP8>
+constexpr bool tcw_layout_ok() {
+    using TL = TcwLayout<FP8>;
+    return TL::kSmem <= 227 * 1024 && TL::kOffP % 1024 == 0 && TL::kOffK % 1024 == 0 && TL::kOffV % 1024 == 0 &&
+           TL::kOffStg % 1024 == 0 && TL::kOffQ % 1024 == 0;
+}
+static_assert(tcw_layout_ok<false>() && tcw_layout_ok<true>(), "many-row tensor-core layout");
 
 // Split of the HCA attention: CTAs per (request, KV head), so that all
 // CTAs fit in one wave at two per SM.

@@ -116,6 +116,10 @@ WORKLOADS = {
     "chunk16_fp8_512k": Workload("chunk16_fp8_512k", batch=4, q_tokens=16, num_q_heads=32,
                                  num_kv_heads=8, seq_len=524288, kv_fp8=True, structure="zipf",
                                  mode="topk", max_ratio=0.12, seed=1239),
+    # the fp8 chunk shape at 128K context: small enough for detailed profiling
+    "chunk16_fp8_128k": Workload("chunk16_fp8_128k", batch=4, q_tokens=16, num_q_heads=32,
+                                 num_kv_heads=8, seq_len=131072, kv_fp8=True, structure="zipf",
+                                 mode="topk", max_ratio=0.12, seed=1242),
 }
 
 BENCH_WORKLOAD = "decode_128k_b8"

@@ -218,9 +218,11 @@ size_t spattn_decode_workspace_size(const spattn_dims *dims, const spattn_params
  * fp32 accumulation; split-KV partials merged by their log-sum-exp).
  * A row with no visible token is all zeros.  sel_idx / sel_count as written
  * by spattn_select (any ascending or unordered list of distinct ids works).
- * bf16 caches with Tq * Hq / Hkv <= 16 run on the tensor cores (tcgen05,
- * probabilities entered as bf16 hi + lo parts); fp8 caches and larger row
- * counts on CUDA cores.
+ * Both kernels run on the tensor cores (tcgen05, probabilities entered as
+ * bf16 hi + lo parts): bf16 caches with Tq * Hq / Hkv <= 16 with the tokens
+ * of a block on M; fp8 caches (codes widened to bf16 in shared memory, the
+ * scales applied to the scores and the weights) and larger row counts with
+ * the query rows on M.
  */
 spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_params *params,
                                      const void *q, const void *k_cache, const void *v_cache,
@@ -265,9 +267,8 @@ spattn_status spattn_decode_selected_lse(const spattn_dims *dims, const spattn_p
  * exits).  Arguments, layouts and results are those of
  * spattn_decode_selected; dims whose partial results need more than 16 MiB
  * ((320 + B * Hkv) x R x (Tq * Hq / Hkv) x (d + 2) x 4 bytes, R = 4 records
- * per slot on the tensor-core path -- bf16 caches with Tq * Hq / Hkv <= 16 --
- * and 1 otherwise) are rejected with SPATTN_ERR_UNSUPPORTED before anything
- * is enqueued.  No allocation call is
+ * per slot for bf16 caches with Tq * Hq / Hkv <= 16, 1 otherwise) are
+ * rejected with SPATTN_ERR_UNSUPPORTED before anything is enqueued.  No allocation call is
  * made.  The first call on each device looks up the array's device address
  * (a host-side CUDA runtime call), so make that first call before any stream
  * capture.  Every call on a device shares the one array and leaves its

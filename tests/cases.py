@@ -33,5 +33,11 @@ CHUNK2_ANCHOR = Workload("chunk2_anchor", batch=2, q_tokens=2, num_q_heads=16, n
                          seq_len=64 * 90 + 40, structure="planted", n_planted=8, mode="topp_anchor",
                          top_p=0.8, min_ratio=0.05, max_ratio=0.25, seed=19)
 
+# bf16 cache with 64 query rows per KV head (8 tokens x 8 heads): the
+# many-row tensor-core kernel
+CHUNK8_WIDE = Workload("chunk8_wide", batch=2, q_tokens=8, num_q_heads=16, num_kv_heads=2,
+                       seq_len=64 * 70 + 21, structure="zipf", mode="topp", top_p=0.9,
+                       max_ratio=0.2, seed=20)
+
 SMALL_CASES = [WORKLOADS["tiny_4k_gqa4"], SMALL_TOPP, SMALL_FP8_CHUNK, SMALL_RAGGED, GQA8_TOPP,
-               MQA16_TOPK, CHUNK16_FP8, CHUNK2_TOPP, GQA4_128K_SMALL, SMALL_ANCHOR, CHUNK2_ANCHOR]
+               MQA16_TOPK, CHUNK16_FP8, CHUNK2_TOPP, GQA4_128K_SMALL, SMALL_ANCHOR, CHUNK2_ANCHOR, CHUNK8_WIDE]
