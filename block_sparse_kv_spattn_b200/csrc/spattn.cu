@@ -56,8 +56,9 @@ spattn_status cuda_ok(cudaError_t e, const char *what) {
     return fail(SPATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// Upper bound on persistent attention CTAs (2 per SM); the workspace is sized
-// for it so that workspace sizes need no device query.
+// Upper bound on persistent attention CTAs (one per SM, for devices of up to
+// 320 SMs); the workspace is sized for it so that workspace sizes need no
+// device query.
 constexpr int kMaxAttnCtas = 2 * 160;
 constexpr size_t kAlign = 256;
 
@@ -149,13 +150,6 @@ bool uses_tc(const spattn_dims *d) { return d->kv_dtype == SPATTN_KV_BF16 && row
 // Partial records per (CTA, unit) slot: one per softmax warp (attn_tc), one
 // (attn_tcw).
 int records_per_slot(const spattn_dims *d) { return uses_tc(d) ? kTcWarpSlots : 1; }
-
-int rg_of(int rows) {
-    const int rg = (rows + 3) / 4;
-    int p = 1;
-    while (p < rg) p <<= 1;
-    return p;
-}
 
 // Per-device caches (SM count; which kernels have their shared-memory limit
 // raised).  Guarded by one mutex: these are host-side set-up calls only.
@@ -346,38 +340,6 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
                    "select launch");
 }
 
-std::map<std::pair<int, const void *>, int> g_occ;
-
-// Resident CTAs per SM of a kernel (queried once per device), capped at
-// `want`: the persistent grid is sized to what can actually be resident.
-spattn_status resident_ctas(const void *func, int threads, int smem, int want, int *out) {
-    int dev;
-    SP_TRY(cuda_ok(cudaGetDevice(&dev), "cudaGetDevice"));
-    std::lock_guard<std::mutex> lk(g_mu);
-    auto it = g_occ.find({dev, func});
-    if (it == g_occ.end()) {
-        int n = 0;
-        SP_TRY(cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem),
-                       "cudaOccupancyMaxActiveBlocksPerMultiprocessor"));
-        it = g_occ.emplace(std::make_pair(dev, func), n).first;
-    }
-    *out = std::max(1, std::min(want, it->second));
-    return SPATTN_OK;
-}
-
-template <int RG, bool FP8>
-spattn_status launch_attn_t(AttnArgs &a, int sms, cudaStream_t st, int *ctas_out) {
-    const int smem = attn_smem_bytes(FP8, RG);
-    const void *fn = (const void *)attn_kernel<RG, FP8>;
-    SP_TRY(ensure_smem(fn, smem));
-    int per_sm;
-    SP_TRY(resident_ctas(fn, kAttnThreads, smem, attn_ctas_per_sm(RG), &per_sm));
-    const int ctas = std::min(kMaxAttnCtas, sms * per_sm);
-    *ctas_out = ctas;
-    return cuda_ok(launch(attn_kernel<RG, FP8>, dim3(ctas), dim3(kAttnThreads), smem, st, a),
-                   "attention launch");
-}
-
 // cuTensorMapEncodeTiled, reached through the runtime's driver entry point.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -475,18 +437,6 @@ spattn_status launch_attn_tc(AttnArgs &a, const void *k_cache, const void *v_cac
     return launch_attn_tc_t<16>(a, kmap, vmap, sms, st, ctas_out);
 }
 
-template <bool FP8>
-spattn_status launch_attn_rg(int rg, AttnArgs &a, int sms, cudaStream_t st, int *ctas) {
-    switch (rg) {
-        case 1: return launch_attn_t<1, FP8>(a, sms, st, ctas);
-        case 2: return launch_attn_t<2, FP8>(a, sms, st, ctas);
-        case 4: return launch_attn_t<4, FP8>(a, sms, st, ctas);
-        case 8: return launch_attn_t<8, FP8>(a, sms, st, ctas);
-        case 16: return launch_attn_t<16, FP8>(a, sms, st, ctas);
-    }
-    return fail(SPATTN_ERR_UNSUPPORTED, "row groups %d", rg);
-}
-
 spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, const void *q,
                                const void *k_cache, const void *v_cache, const float *k_scale,
                                const float *v_scale, const int32_t *bt, const int32_t *sl,
@@ -494,7 +444,6 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
                                float *lse, char *ws, const DecodeLayout &L, cudaStream_t st) {
     const bool fp8 = d->kv_dtype == SPATTN_KV_FP8_E4M3;
     const int rows = rows_of(d);
-    const int rg = rg_of(rows);
     int sms;
     SP_TRY(sm_count(&sms));
     AttnArgs a;
@@ -594,11 +543,6 @@ spattn_status noalloc_scratch(void **out) {
     return SPATTN_OK;
 }
 
-// The attention kernel's shared-memory regions are 16-byte aligned and the
-// two-CTA-per-SM shapes fit two CTAs (228 KiB per SM, 1 KiB reserved each).
-static_assert(attn_off_pbuf(false, 1) % 16 == 0 && attn_off_pbuf(true, 16) % 16 == 0, "layout");
-static_assert(2 * (attn_smem_bytes(false, 1) + 1024) <= 228 * 1024, "two CTAs per SM at one row group");
-static_assert(attn_smem_bytes(false, 16) <= 227 * 1024, "one CTA per SM at sixteen row groups");
 template <int RQ>
 constexpr bool tc_layout_ok() {
     using TL = TcLayout<RQ>;
