@@ -111,6 +111,16 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes) {
     return (nz * 0x3800u + mag) | (h2 & 0x80008000u);
 }
 
+// 2^x by the hardware approximation (relative error ~2^-22), results below
+// the normal range flushed to zero: a weight that small is below the fp32
+// resolution of the row sum, which is at least 1 (the maximum's own weight)
+// or, before the row's first visible score, exactly 0.
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // 64 consecutive 32-bit TMEM columns of this thread's lane, one load.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
     uint32_t r[64];
@@ -555,7 +565,7 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
             float ps = 0.f;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const float p0 = exp2f(x[2 * e] - mu), p1 = exp2f(x[2 * e + 1] - mu);
+                const float p0 = ex2_ftz(x[2 * e] - mu), p1 = ex2_ftz(x[2 * e + 1] - mu);
                 ps += p0 + p1;
                 // hi = p with its low 16 bits cleared (a bf16 value), lo = the
                 // exact fp32 remainder, truncated the same way: the pair keeps
