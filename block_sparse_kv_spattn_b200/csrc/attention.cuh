@@ -59,6 +59,14 @@ __device__ __forceinline__ int unit_count(const AttnArgs &a, int u) {
 __host__ __device__ __forceinline__ int cta_of(int64_t x, int64_t W, int C) {
     return (int)(((x + 1) * C + W - 1) / W) - 1;
 }
+// A 16-byte global load issued here (the compiler may not sink it towards
+// its use), so that several can be in flight before their results matter.
+__device__ __forceinline__ float4 ld_f4_now(const float *p) {
+    float4 v;
+    asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+
 struct MergeArgs {
     const float *part_o;
     const float *part_ml;
@@ -127,17 +135,34 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
         // wrote only if it took a tile
         const int c_lo = cta_of(pre, W, a.ctas), c_hi = cta_of(pre + cnt - 1, W, a.ctas);
         const int nrec = (c_hi - c_lo + 1) * a.wslots;
-        // batches of 32 records, one per lane, merged online: the lanes load
-        // their records' (m, l) together, then the row's O of every record of
-        // the batch is loaded in one unrolled run (no record waits on another)
+        // batches of 32 records, one per lane, merged online.  A written
+        // record's row is finite even when its maximum is -inf (zero weights
+        // over zeroed unfilled slots), so the rows of the batch's first 16
+        // records are loaded together with the maxima, before the weights
+        // are known; a record that was not written reads a written one
+        // (weight 0).
         for (int x0 = 32 * warp; x0 < nrec; x0 += 32 * nw) {
             const int64_t r = x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
+            const unsigned written = __ballot_sync(0xffffffffu, r >= 0);
+            if (!written) continue;   // uniform
+            // (every lane takes part in the shuffle, then picks)
+            const int64_t rfirst = __shfl_sync(0xffffffffu, r, __ffs(written) - 1);
+            const int64_t rr = r >= 0 ? r : rfirst;
+            const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
+            float4 o16[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int64_t re = __shfl_sync(0xffffffffu, rr, e);
+                o16[e] = e < n_here ? ld_f4_now(a.part_o + (re * a.rows + row) * kHeadDim + lane * 4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
             float2 ml = make_float2(-INFINITY, 0.f);
             if (r >= 0) ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
             const float Mb = fmaxf(M, warp_max(ml.x));
             const unsigned valid = __ballot_sync(0xffffffffu, r >= 0 && ml.x != -INFINITY);
-            if (Mb == -INFINITY || !valid) continue;   // uniform: nothing to add
-            if (Mb != M) {   // uniform: rescale what is summed so far
+            // (no early exit here: the rows above stay in flight; a batch
+            // with nothing valid adds zero weights)
+            if (valid && Mb != M) {   // uniform: rescale what is summed so far
                 const float f = M == -INFINITY ? 0.f : exp2f(M - Mb);
                 acc.x *= f;
                 acc.y *= f;
@@ -151,12 +176,16 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
                 w = exp2f(ml.x - M);
                 lsum = fmaf(w, ml.y, lsum);
             }
-            // records without weight read the first valid one (weight 0)
-            const int64_t rfirst = __shfl_sync(0xffffffffu, r, __ffs(valid) - 1);
-            const int64_t rr = ((valid >> lane) & 1u) ? r : rfirst;
-            const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float we = __shfl_sync(0xffffffffu, w, e);
+                acc.x = fmaf(we, o16[e].x, acc.x);
+                acc.y = fmaf(we, o16[e].y, acc.y);
+                acc.z = fmaf(we, o16[e].z, acc.z);
+                acc.w = fmaf(we, o16[e].w, acc.w);
+            }
 #pragma unroll 16
-            for (int e = 0; e < n_here; ++e) {
+            for (int e = 16; e < n_here; ++e) {
                 const float we = __shfl_sync(0xffffffffu, w, e);
                 const int64_t re = __shfl_sync(0xffffffffu, rr, e);
                 const float4 o = reinterpret_cast<const float4 *>(a.part_o + (re * a.rows + row) * kHeadDim)[lane];
