@@ -48,7 +48,8 @@ from block_sparse_kv_spattn_b200.workloads import BENCH_WORKLOAD, WORKLOADS, mak
 METRIC = "selected-KV HBM GB/s (% of ~8 TB/s) and decode queries/s at 128K ctx, 1 B200"
 FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
-ATTN_SOURCES = ["common.cuh", "attention.cuh", "tcgen05.cuh", "attention_tc.cuh", "attention_tcw.cuh"]
+# the sources of the kernel the traffic capture covers (attn_tc_kernel)
+ATTN_SOURCES = ["common.cuh", "attention.cuh", "tcgen05.cuh", "attention_tc.cuh"]
 
 
 def _peaks():
@@ -78,15 +79,16 @@ def attn_label(w) -> str:
             f"+ merge_kernel, one decode_selected call)")
 
 
-def measured_traffic(units_in_launch: float):
+def measured_traffic(w, units_in_launch: float):
     """DRAM bytes per launch of the attention kernel from the committed ncu
-    capture, scaled to this launch; None if the kernel changed since."""
+    capture, scaled to this launch; None if this workload runs another
+    kernel or the kernel's sources changed since."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except Exception:
         return None
-    if t.get("source_sha") != attn_source_hash():
+    if t.get("kernel", "") not in attn_label(w) or t.get("source_sha") != attn_source_hash():
         return None
     return t["dram_bytes_per_launch"] * units_in_launch / t["units_per_launch"]
 
@@ -360,7 +362,7 @@ def run_native(args, rank, world, local_rank):
     attn_ms_mean = attn_total_ms / K
     attn_bytes = bts["kv"] + bts["q"] + bts["out"]     # one rank's launch
     achieved = attn_bytes / (attn_ms_mean * 1e-3) / 1e9
-    traffic = measured_traffic(bts["kept_block_heads"])
+    traffic = measured_traffic(w, bts["kept_block_heads"])
     queries = B * Tq * world / (ms_per_step * 1e-3)
     e2e_value = all_bytes / (e2e_total_ms / K * 1e-3) / 1e9
     line = {

@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libspattn.so")
 SOURCES = ["spattn.cu"]
 DEPS = ["common.cuh", "compress.cuh", "scores.cuh", "select.cuh", "attention.cuh", "tcgen05.cuh",
-        "attention_tc.cuh", "attention_tcw.cuh", "hca.cuh", "exports.map"]
+        "attention_tc.cuh", "attention_tcw.cuh", "merge.cuh", "hca.cuh", "exports.map"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,0 +1,185 @@
+// merge.cuh -- the split merge: one softmax per output row from the partial
+// records the attention kernels write per (CTA, unit) slot.
+//
+// "CSA + HCA 混合注意力机制" §4.4 step 4 (one softmax over the selected entries):
+// a unit whose kept blocks were split over several CTAs gets partial results
+// (base-2 maximum m_s, sum l_s, unnormalised output o_s per row), combined as
+// out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+#pragma once
+
+#include "attention.cuh"
+
+namespace spattn {
+
+// A 16-byte global load issued here (the compiler may not sink it towards
+// its use), so that several can be in flight before their results matter.
+__device__ __forceinline__ float4 ld_f4_now(const float *p) {
+    float4 v;
+    asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+
+struct MergeArgs {
+    const float *part_o;
+    const float *part_ml;
+    const int32_t *sel_count;
+    float *out;                 // [B][Tq][Hq][D]
+    float *lse;                 // nullable: [B][Tq][Hq], ln of the row's sum of exp(logit)
+    int batch, tq, hq, hkv, group, rows, units, max_sel, ctas;
+    int wslots;                 // partial records per (CTA, unit): 1, 2 (hi / lo parts) or 4 (per softmax warp)
+    int pairs;                  // 4 records: warp w's pair w / 2 took only tiles of its parity
+};
+
+constexpr int kMergeMaxWarps = 8;   // warps per output row, for units split over many CTAs
+
+// Record x of a unit's candidate list (CTA c_lo + x / wslots, warp x %
+// wslots), or -1 if it was not written: the CTA's range misses the unit's
+// [pre, pre + cnt) part (only when W < C), or, with one record per
+// tensor-core softmax warp, the warp's pair took none of the CTA's tiles of
+// the unit (pair p takes CTA-local tile indices of parity p).
+__device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int x, int c_lo, int unit, int64_t pre, int cnt,
+                                                int64_t W) {
+    const int cc = c_lo + x / a.wslots, w = x % a.wslots;
+    const int64_t lo_c = W * cc / a.ctas, hi_c = W * (cc + 1) / a.ctas;
+    const int64_t ia = (pre > lo_c ? pre : lo_c) - lo_c;
+    const int64_t ib = (pre + cnt < hi_c ? pre + cnt : hi_c) - lo_c;
+    if (ib <= ia) return -1;
+    if (a.pairs && ib - ia < 2 && (ia & 1) != (w >> 1)) return -1;
+    return ((int64_t)cc + unit) * a.wslots + w;
+}
+
+// One CTA per output row (b, t, query head): out = sum_s 2^(m_s - M) o_s /
+// sum_s 2^(m_s - M) l_s over the partial records of the row's unit: slot
+// c + unit for each CTA c whose range meets the unit's part of the sequence
+// (with wslots = 4, record w of that slot for each softmax warp w whose pair
+// took one of the CTA's tiles of the unit: pair w / 2 takes the tiles with
+// CTA-local index of its parity).  The CTA's warps take batches of 32
+// records in turn (a unit split over many CTAs has hundreds) and are
+// combined through shared memory.  A unit with nothing kept gets a zero row.
+__global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a) {
+    __shared__ float s_m[kMergeMaxWarps], s_l[kMergeMaxWarps];
+    __shared__ float4 s_acc[kMergeMaxWarps][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int64_t grow = blockIdx.x;
+    const int i = (int)(grow % a.hq);
+    const int t = (int)((grow / a.hq) % a.tq);
+    const int b = (int)(grow / ((int64_t)a.hq * a.tq));
+    const int h = i / a.group, g = i % a.group;
+    const int unit = b * a.hkv + h;
+    const int row = t * a.group + g;
+    // prefix of the unit in the concatenated sequence, and the total W
+    int64_t pre = 0, W = 0;
+    for (int u = lane; u < a.units; u += 32) {
+        const int cnt = min(max(a.sel_count[u], 0), a.max_sel);
+        W += cnt;
+        if (u < unit) pre += cnt;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        pre += __shfl_xor_sync(0xffffffffu, pre, o);
+        W += __shfl_xor_sync(0xffffffffu, W, o);
+    }
+    const int cnt = min(max(a.sel_count[unit], 0), a.max_sel);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.f, M = -INFINITY;
+    if (cnt > 0) {
+        // records r = (slot * wslots + w) that were written: CTAs with an
+        // empty range (only when W < C) wrote none; with wslots = 4 a pair
+        // wrote only if it took a tile
+        const int c_lo = cta_of(pre, W, a.ctas), c_hi = cta_of(pre + cnt - 1, W, a.ctas);
+        const int nrec = (c_hi - c_lo + 1) * a.wslots;
+        // batches of 32 records, one per lane, merged online.  A written
+        // record's row is finite even when its maximum is -inf (zero weights
+        // over zeroed unfilled slots), so the rows of the batch's first 16
+        // records are loaded together with the maxima, before the weights
+        // are known; a record that was not written reads a written one
+        // (weight 0).
+        for (int x0 = 32 * warp; x0 < nrec; x0 += 32 * nw) {
+            const int64_t r = x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
+            const unsigned written = __ballot_sync(0xffffffffu, r >= 0);
+            if (!written) continue;   // uniform
+            // (every lane takes part in the shuffle, then picks)
+            const int64_t rfirst = __shfl_sync(0xffffffffu, r, __ffs(written) - 1);
+            const int64_t rr = r >= 0 ? r : rfirst;
+            const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
+            float4 o16[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int64_t re = __shfl_sync(0xffffffffu, rr, e);
+                o16[e] = e < n_here ? ld_f4_now(a.part_o + (re * a.rows + row) * kHeadDim + lane * 4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            float2 ml = make_float2(-INFINITY, 0.f);
+            if (r >= 0) ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
+            const float Mb = fmaxf(M, warp_max(ml.x));
+            const unsigned valid = __ballot_sync(0xffffffffu, r >= 0 && ml.x != -INFINITY);
+            // (no early exit here: the rows above stay in flight; a batch
+            // with nothing valid adds zero weights)
+            if (valid && Mb != M) {   // uniform: rescale what is summed so far
+                const float f = M == -INFINITY ? 0.f : exp2f(M - Mb);
+                acc.x *= f;
+                acc.y *= f;
+                acc.z *= f;
+                acc.w *= f;
+                lsum *= f;
+                M = Mb;
+            }
+            float w = 0.f;
+            if ((valid >> lane) & 1u) {
+                w = exp2f(ml.x - M);
+                lsum = fmaf(w, ml.y, lsum);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float we = __shfl_sync(0xffffffffu, w, e);
+                acc.x = fmaf(we, o16[e].x, acc.x);
+                acc.y = fmaf(we, o16[e].y, acc.y);
+                acc.z = fmaf(we, o16[e].z, acc.z);
+                acc.w = fmaf(we, o16[e].w, acc.w);
+            }
+#pragma unroll 16
+            for (int e = 16; e < n_here; ++e) {
+                const float we = __shfl_sync(0xffffffffu, w, e);
+                const int64_t re = __shfl_sync(0xffffffffu, rr, e);
+                const float4 o = reinterpret_cast<const float4 *>(a.part_o + (re * a.rows + row) * kHeadDim)[lane];
+                acc.x = fmaf(we, o.x, acc.x);
+                acc.y = fmaf(we, o.y, acc.y);
+                acc.z = fmaf(we, o.z, acc.z);
+                acc.w = fmaf(we, o.w, acc.w);
+            }
+        }
+        lsum = warp_sum(lsum);
+    }
+    if (nw > 1) {
+        // combine the warps: weights 2^(M_w - M)
+        if (lane == 0) {
+            s_m[warp] = M;
+            s_l[warp] = lsum;
+        }
+        s_acc[warp][lane] = acc;
+        __syncthreads();
+        if (warp != 0) return;
+        float Mt = -INFINITY;
+        for (int w = 0; w < nw; ++w) Mt = fmaxf(Mt, s_m[w]);
+        M = Mt;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        lsum = 0.f;
+        if (Mt != -INFINITY)
+            for (int w = 0; w < nw; ++w) {
+                if (s_m[w] == -INFINITY) continue;
+                const float f = exp2f(s_m[w] - Mt);
+                const float4 o = s_acc[w][lane];
+                lsum = fmaf(f, s_l[w], lsum);
+                acc.x = fmaf(f, o.x, acc.x);
+                acc.y = fmaf(f, o.y, acc.y);
+                acc.z = fmaf(f, o.z, acc.z);
+                acc.w = fmaf(f, o.w, acc.w);
+            }
+    }
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    reinterpret_cast<float4 *>(a.out + grow * kHeadDim)[lane] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    // records hold base-2 maxima of the scaled logits: ln sum = (M + log2 l) ln 2
+    if (a.lse && lane == 0) a.lse[grow] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace spattn

@@ -22,6 +22,7 @@
 #include "attention.cuh"
 #include "attention_tc.cuh"
 #include "attention_tcw.cuh"
+#include "merge.cuh"
 #include "hca.cuh"
 
 using namespace spattn;
