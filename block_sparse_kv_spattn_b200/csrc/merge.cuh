@@ -26,7 +26,7 @@ struct MergeArgs {
     float *out;                 // [B][Tq][Hq][D]
     float *lse;                 // nullable: [B][Tq][Hq], ln of the row's sum of exp(logit)
     int batch, tq, hq, hkv, group, rows, units, max_sel, ctas;
-    int wslots;                 // partial records per (CTA, unit): 1, 2 (hi / lo parts) or 4 (per softmax warp)
+    int wslots;                 // partial records per (CTA, unit): 1 (attn_tcw) or 4 (one per attn_tc softmax warp)
     int pairs;                  // 4 records: warp w's pair w / 2 took only tiles of its parity
 };
 
@@ -37,8 +37,8 @@ constexpr int kMergeMaxWarps = 8;   // warps per output row, for units split ove
 // [pre, pre + cnt) part (only when W < C), or, with one record per
 // tensor-core softmax warp, the warp's pair took none of the CTA's tiles of
 // the unit (pair p takes CTA-local tile indices of parity p).
-__device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int x, int c_lo, int unit, int64_t pre, int cnt,
-                                                int64_t W) {
+__host__ __device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int x, int c_lo, int unit,
+                                                         int64_t pre, int cnt, int64_t W) {
     const int cc = c_lo + x / a.wslots, w = x % a.wslots;
     const int64_t lo_c = W * cc / a.ctas, hi_c = W * (cc + 1) / a.ctas;
     const int64_t ia = (pre > lo_c ? pre : lo_c) - lo_c;
