@@ -28,6 +28,8 @@ constexpr int kScoreThreads = 128;
 // Blocks per CTA: small CTAs (many resident per SM, many loads in flight)
 // unless the query rows make the per-CTA q-bar prologue heavy.
 __host__ __device__ constexpr int score_blocks_per_cta(int rows) { return rows <= 16 ? 16 : 64; }
+static_assert(score_blocks_per_cta(1) <= kScoreThreads && score_blocks_per_cta(64) <= kScoreThreads,
+              "one block-table entry per thread");
 
 // Sum of v[0..7] over the 32 lanes, scattered: afterwards lane l holds the
 // full sum of element (l >> 2) & 7.  Butterfly halving at offsets 16, 8, 4
@@ -76,26 +78,15 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     // this grid's completion before it reads the scores
     asm volatile("griddepcontrol.launch_dependents;");
 
+    // this thread's block-table entry (one block of the CTA's range per
+    // thread), loaded beside the length instead of after it: which entries
+    // count is decided once the length is known
+    const int tj = threadIdx.x, tblk = j0 + tj;
+    const int page_raw =
+        (tj < a.bpc && tblk < a.max_blocks) ? a.block_table[(int64_t)b * a.max_blocks + tblk] : -1;
     int L = a.seq_lens[b];
-    if (L < 0 || L > a.max_blocks * kBlock) {
-        if (threadIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
-        L = 0;
-    }
-    const int nb = (L + kBlock - 1) / kBlock;
-
-    // 1. page ids of the middle blocks, and group-mean query rows (8 columns per task)
-    for (int jj = threadIdx.x; jj < a.bpc; jj += kScoreThreads) {
-        const int j = j0 + jj;
-        int page = -1;
-        if (j < a.max_blocks && j < nb && (a.anchors || (j >= a.sink && j < nb - a.local))) {
-            page = a.block_table[(int64_t)b * a.max_blocks + j];
-            if (page < 0 || page >= a.num_pages) {
-                flag(SPATTN_DEV_BAD_PAGE);
-                page = -1;
-            }
-        }
-        pages[jj] = page;
-    }
+    // 1. group-mean query rows (8 columns per task); their loads, the length
+    // and the table entry are in flight together
     for (int task = threadIdx.x; task < rows * (kHeadDim / 8); task += kScoreThreads) {
         const int c8 = task % (kHeadDim / 8), th = task / (kHeadDim / 8);
         const int hh = th % HKV, t = th / HKV;
@@ -120,9 +111,27 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
         dst[0] = make_float4(s[0] / G, s[1] / G, s[2] / G, s[3] / G);
         dst[1] = make_float4(s[4] / G, s[5] / G, s[6] / G, s[7] / G);
     }
+    if (L < 0 || L > a.max_blocks * kBlock) {
+        if (threadIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
+        L = 0;
+    }
+    const int nb = (L + kBlock - 1) / kBlock;
+
+    // 2. page ids of the middle blocks, once the length is known
+    if (tj < a.bpc) {
+        int page = -1;
+        if (tblk < a.max_blocks && tblk < nb && (a.anchors || (tblk >= a.sink && tblk < nb - a.local))) {
+            page = page_raw;
+            if (page < 0 || page >= a.num_pages) {
+                flag(SPATTN_DEV_BAD_PAGE);
+                page = -1;
+            }
+        }
+        pages[tj] = page;
+    }
     __syncthreads();
 
-    // 2. lane owns columns [4*lane, 4*lane+4) of every KV head's kbar row
+    // 3. lane owns columns [4*lane, 4*lane+4) of every KV head's kbar row
     constexpr int HPC = HKV < 8 ? HKV : 8;      // heads per 8-value chunk
     constexpr int TPC = 8 / HPC;                // tokens per chunk
     for (int jb = warp; jb < a.bpc; jb += NW * BIF) {
@@ -190,7 +199,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     }
     __syncthreads();
 
-    // 3. coalesced store of the tile
+    // 4. coalesced store of the tile
     for (int idx = threadIdx.x; idx < rows * a.bpc; idx += kScoreThreads) {
         const int jj = idx % a.bpc, r = idx / a.bpc;
         const int j = j0 + jj;

@@ -322,10 +322,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     }
     const int bh = blockIdx.x;
     const int b = bh / a.hkv, h = bh % a.hkv;
-    // launched early (programmatic dependent launch): wait for the previous
-    // grid in the stream (the scoring) to complete before reading anything
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // launched early (programmatic dependent launch): the length is an input
+    // the scoring does not write, so its load goes out now; the scores are
+    // read only after the previous grid in the stream (the scoring) completed
     int L = a.seq_lens[b];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // the first token's score row into L1
     {
         const float *row0 = a.scores + ((int64_t)b * a.tq * a.hkv + h) * a.max_blocks;
