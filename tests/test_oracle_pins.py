@@ -332,6 +332,28 @@ def test_sparse_attention_equals_masked_sdpa(w):
     np.testing.assert_allclose(res["out"], ref, rtol=1e-10, atol=1e-12)
 
 
+LONG_CHUNK = Workload("long_chunk", batch=1, q_tokens=200, num_q_heads=8, num_kv_heads=2,
+                      seq_len=64 * 20 + 9, structure="zipf", mode="topk", max_ratio=0.3, seed=31)
+
+
+def test_long_chunk_is_causal_everywhere():
+    """A chunk longer than the local window (200 tokens against 2 x 64): its
+    early tokens must not see the later tokens of middle blocks either, so the
+    causal mask applies to every kept block, selected or all."""
+    inp = make_inputs(LONG_CHUNK)
+    res = run_oracle(inp, params=params_of(LONG_CHUNK, **SELECT_ALL))
+    np.testing.assert_allclose(res["out"], _sdpa_reference(inp), rtol=1e-10, atol=1e-12)
+    res = run_oracle(inp)
+    nbmax = inp["max_blocks"]
+
+    def keep(b, h):
+        m = torch.zeros(nbmax, dtype=torch.bool)
+        m[torch.from_numpy(res["sel_idx"][b, h, :res["sel_count"][b, h]]).long()] = True
+        return m
+
+    np.testing.assert_allclose(res["out"], _sdpa_reference(inp, keep), rtol=1e-10, atol=1e-12)
+
+
 def test_two_token_closed_form():
     """One request of 2 tokens, one head: out = (e^a v1 + e^b v2) / (e^a + e^b)."""
     w = Workload("two", batch=1, q_tokens=1, num_q_heads=1, num_kv_heads=1, seq_len=2,
