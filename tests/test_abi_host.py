@@ -138,3 +138,25 @@ def test_hca_entry_points_validate_on_the_host(lib):
     st = lib.spattn_decode_selected_lse(ctypes.byref(d), ctypes.byref(p.c()), dummy, dummy, dummy, None,
                                         None, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 16, None)
     assert st == 4
+
+
+@pytest.mark.parametrize("kw,records", [
+    (dict(), 4),                                                  # bf16, 4 rows: one record per softmax warp
+    (dict(q_tokens=4, num_q_heads=16, num_kv_heads=2), 1),        # 32 rows: the many-row kernel, one record
+    (dict(kv_dtype=1), 1),                                        # fp8: the many-row kernel
+])
+def test_workspace_size_is_the_documented_layout(lib, kw, records):
+    """Split-KV partials (C_max + B * Hkv) x R records of rows x (d + 2)
+    fp32, C_max = 320, each part 256-byte aligned; plus the scores (B x Tq x
+    Hkv x max_blocks fp32) when spattn_decode keeps them in the workspace."""
+    d = _dims(**kw)
+    p = spattn.Params(top_k=4)
+
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    rows = d.q_tokens * d.num_q_heads // d.num_kv_heads
+    slots = (320 + d.batch * d.num_kv_heads) * records
+    scores = up(d.batch * d.q_tokens * d.num_kv_heads * d.max_blocks_per_seq * 4)
+    want = scores + up(slots * rows * 128 * 4) + up(slots * rows * 2 * 4)
+    assert lib.spattn_decode_workspace_size(ctypes.byref(d), ctypes.byref(p.c())) == want
