@@ -4,7 +4,8 @@ arrives on, tests/native/wait_timeout.cu, compiled from the kernels' own
 header); it must give up after its limit, report SPATTN_DEV_WAIT_TIMEOUT in
 the device status word, end the kernel normally, and leave the context
 usable.  Bad data found on the device is reported the same way: a selected
-block past the request's end is skipped and flagged, never trapped."""
+block past the request's end is skipped and flagged, never trapped.
+(Named so that pytest collects it after the parity tests.)"""
 import os
 import subprocess
 

@@ -2,7 +2,8 @@
 (block scores, selection, output rows, log-sum-exp) is handed to the library
 as the middle of a larger allocation whose two ends hold a sentinel bit
 pattern; after the calls the ends must be unchanged, on both attention
-kernels (bf16 decode, fp8 chunk, many-row bf16) and the HCA branch."""
+kernels (bf16 decode, fp8 chunk, many-row bf16) and the HCA branch.
+(Named so that pytest collects it after the parity tests.)"""
 import pytest
 import torch
 
