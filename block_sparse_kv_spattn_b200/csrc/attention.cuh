@@ -35,6 +35,12 @@ struct AttnArgs {
     float *part_ml;             // [(C + units) * records per slot][rows][2]
     int tq, hq, hkv, group, rows, units, num_pages, max_blocks, max_sel;
     float qscale;               // sm_scale * log2(e)
+    // merge inside the attention kernel (attn_tc_kernel only): the last warp
+    // to finish a unit's tiles merges its records at the end of its CTA
+    int fuse;
+    int32_t *arrive;            // [units] tiles-per-warp arrivals, zero between calls
+    float *out;                 // [B][Tq][Hq][D]
+    float *lse;                 // nullable: [B][Tq][Hq]
 };
 
 struct StageMeta {
@@ -43,7 +49,7 @@ struct StageMeta {
     int unit;     // b * Hkv + h
     int flags;    // kFirst | kLast | kEnd
     int seg;      // segment id within the CTA (tensor-core kernel)
-    int unused1;
+    int pre;      // first index of the unit in the concatenated kept lists
     int qslot;    // query slot holding the segment's query rows
     int pad;
 };

@@ -322,9 +322,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     }
     const int bh = blockIdx.x;
     const int b = bh / a.hkv, h = bh % a.hkv;
-    // launched early (programmatic dependent launch): the length is an input
-    // the scoring does not write, so its load goes out now; the scores are
-    // read only after the previous grid in the stream (the scoring) completed
+    // When launched early behind the scoring grid of the same decode call
+    // (programmatic dependent launch), the length, which the scoring does not
+    // write, is loaded now; the scores are read only after the scoring grid
+    // completed.  Launched normally (standalone selection), the wait returns
+    // at once.
     int L = a.seq_lens[b];
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the first token's score row into L1

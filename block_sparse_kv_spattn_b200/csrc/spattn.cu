@@ -191,18 +191,28 @@ spattn_status sm_count(int *out) {
 constexpr int kMaxSmem = 227 * 1024;
 
 struct DecodeLayout {
-    size_t scores_off, scores_bytes, part_o_off, part_ml_off, total;
+    size_t arrive_off, scores_off, scores_bytes, part_o_off, part_ml_off, total;
 };
 
-// Workspace: [scores] | partial outputs | partial (max, sum).  (C_max +
-// units) slots of `rows` query rows, records_per_slot() records per slot.
+// Arrival counts of the merge inside the attention kernel: a fixed region
+// at the start of every decode workspace (so that it stays in place
+// whatever the dims of the call), zero between calls.
+constexpr int kArriveUnits = 8192;
+constexpr size_t kArriveBytes = kArriveUnits * sizeof(int32_t);
+constexpr int kFuseMaxRecords = 64;   // records per unit, on average, up to which the kernel merges
+
+// Workspace: arrival counts | [scores] | partial outputs | partial (max,
+// sum).  (C_max + units) slots of `rows` query rows, records_per_slot()
+// records per slot.
 DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
     DecodeLayout L{};
     const int64_t units = (int64_t)d->batch * d->num_kv_heads;
     const int64_t slots = (kMaxAttnCtas + units) * records_per_slot(d);
     const int64_t rows = rows_of(d);
     size_t off = 0;
-    L.scores_off = 0;
+    L.arrive_off = 0;
+    off += align_up(kArriveBytes);
+    L.scores_off = off;
     L.scores_bytes = with_scores ? align_up((size_t)d->batch * d->q_tokens * d->num_kv_heads *
                                             d->max_blocks_per_seq * sizeof(float))
                                  : 0;
@@ -302,8 +312,17 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     return cuda_ok(e, "block_scores launch");
 }
 
+// `early`: launched behind block_scores_kernel of the same call (which
+// releases its dependents at entry), so that the selection's prologue
+// overlaps the scoring.  The prologue reads seq_lens before it waits for the
+// scoring grid; that is safe only when the kernel before it in the stream is
+// that scoring grid (which does not write seq_lens, and which itself started
+// after every earlier kernel had finished).  The standalone spattn_select
+// follows whatever the caller ran last (possibly the kernel that updates
+// seq_lens), so it launches normally.
 spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const float *scores,
-                            const int32_t *sl, int32_t *sel_idx, int32_t *sel_count, cudaStream_t st) {
+                            const int32_t *sl, int32_t *sel_idx, int32_t *sel_count, bool early,
+                            cudaStream_t st) {
     SelectArgs a;
     a.scores = scores;
     a.seq_lens = sl;
@@ -337,7 +356,9 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
     // passes (measured: 512 beat 1024 by 15-25 % on 2K-4K middle blocks)
     const int nm = n_mid_cap(d, p);
     const int threads = nm <= 1024 ? 256 : (nm <= 4096 ? 512 : kSelThreads);
-    return cuda_ok(launch_early(select_kernel, dim3(d->batch * d->num_kv_heads), dim3(threads), smem, st, a),
+    const dim3 grid(d->batch * d->num_kv_heads);
+    return cuda_ok(early ? launch_early(select_kernel, grid, dim3(threads), smem, st, a)
+                         : launch(select_kernel, grid, dim3(threads), smem, st, a),
                    "select launch");
 }
 
@@ -469,14 +490,25 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     a.max_blocks = d->max_blocks_per_seq;
     a.max_sel = d->max_sel;
     a.qscale = sm_scale_of(p) * kLog2e;
-    int ctas = 0;
+    a.out = out;
+    a.lse = lse;
+    a.arrive = reinterpret_cast<int32_t *>(ws + L.arrive_off);
     const bool tc = uses_tc(d);
+    // merge inside the attention kernel when a unit's records are few (a
+    // warp merges a row at a CTA's end) and the counts fit their region
+    {
+        const int64_t recs = ((int64_t)std::min(kMaxAttnCtas, sms) / std::max(1, a.units) + 2) * kTcWarpSlots;
+        a.fuse = tc && a.units <= kArriveUnits && recs <= kFuseMaxRecords &&
+                 (int64_t)a.units * a.max_sel < ((int64_t)1 << 31);
+    }
+    int ctas = 0;
     if (tc)
         SP_TRY(launch_attn_tc(a, k_cache, v_cache, sms, st, &ctas));
     else
         SP_TRY(fp8 ? launch_attn_tcw<true>(a, k_cache, v_cache, sms, st, &ctas)
                    : launch_attn_tcw<false>(a, k_cache, v_cache, sms, st, &ctas));
 
+    if (a.fuse) return SPATTN_OK;
     MergeArgs m;
     m.part_o = a.part_o;
     m.part_ml = a.part_ml;
@@ -706,7 +738,7 @@ spattn_status spattn_select(const spattn_dims *dims, const spattn_params *params
     const int32_t need = required_max_sel(dims, params);
     if (dims->max_sel < need)
         return fail(SPATTN_ERR_INVALID_ARG, "max_sel %d < required %d", dims->max_sel, need);
-    SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count,
+    SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count, false,
                          reinterpret_cast<cudaStream_t>(stream)));
     return ok();
 }
@@ -714,6 +746,15 @@ spattn_status spattn_select(const spattn_dims *dims, const spattn_params *params
 size_t spattn_decode_workspace_size(const spattn_dims *dims, const spattn_params *params) {
     if (check_dims(dims) != SPATTN_OK || check_params(params) != SPATTN_OK) return 0;
     return decode_layout(dims, true).total;
+}
+
+spattn_status spattn_decode_workspace_init(void *workspace, size_t workspace_bytes, spattn_stream_t stream) {
+    if (!workspace || workspace_bytes < kArriveBytes)
+        return fail(SPATTN_ERR_WORKSPACE, "workspace of %zu bytes < %zu (the arrival counts)", workspace_bytes,
+                    kArriveBytes);
+    SP_TRY(cuda_ok(cudaMemsetAsync(workspace, 0, kArriveBytes, reinterpret_cast<cudaStream_t>(stream)),
+                   "workspace init"));
+    return ok();
 }
 
 spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_params *params, const void *q,
@@ -770,8 +811,12 @@ spattn_status spattn_decode_selected_noalloc(const spattn_dims *dims, const spat
     void *scratch = nullptr;
     SP_TRY(noalloc_scratch(&scratch));
     char *ws = static_cast<char *>(scratch);
+    // the arrival counts must start at zero; a completed call leaves them
+    // zero, but one that gave up on a wait may not: clear them every call
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    SP_TRY(cuda_ok(cudaMemsetAsync(ws + L.arrive_off, 0, kArriveBytes, st), "clear scratch counts"));
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
-                            sel_idx, sel_count, out, nullptr, ws, L, reinterpret_cast<cudaStream_t>(stream)));
+                            sel_idx, sel_count, out, nullptr, ws, L, st));
     return ok();
 }
 
@@ -800,7 +845,7 @@ spattn_status spattn_decode(const spattn_dims *dims, const spattn_params *params
     float *scores = scores_out ? scores_out : reinterpret_cast<float *>(ws + L.scores_off);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     SP_TRY(launch_scores(dims, params, q, kbar, block_table, seq_lens, scores, st));
-    SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count, st));
+    SP_TRY(launch_select(dims, params, scores, seq_lens, sel_idx, sel_count, true, st));
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
                             sel_idx, sel_count, out, nullptr, ws, L, st));
     return ok();
