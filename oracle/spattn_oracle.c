@@ -283,7 +283,23 @@ static int anchor_k_max(const spo_params *pr, double a, double hi, double lo, in
 }
 
 /* Number of middle blocks kept for one query row, and the decision margin.
- * a: the anchors' best score (mode 2 only). */
+ * a: the anchors' best score (mode 2 only).
+ *
+ * The decision margin is the distance from the inputs to the nearest point
+ * where the kept set would change, measured on each quantity the decision
+ * is taken on: the score gap across the cut (the worst kept block against
+ * the best dropped one; score units) and, for top-p, the distance of the
+ * threshold p to the nearest prefix mass at which the kept set changes
+ * (probability units).  Top-p keeps the minimal ranked prefix m* with
+ * C_{m*} >= p (C_i: mass of the i best blocks), capped at k_max:
+ *   uncapped (m* <= k_max): p - C_{m*-1} (a lower p reaching C_{m*-1} keeps
+ *     m* - 1 blocks; no such point when m* = 1) and C_{m*} - p (a higher p
+ *     keeps m* + 1; none when m* = n_mid or m* = k_max, where the cap holds
+ *     the set);
+ *   capped (m* > k_max): p - C_{k_max-1} (only a p at or below C_{k_max-1}
+ *     keeps fewer than k_max; none when k_max <= 1); a higher p changes
+ *     nothing.
+ * Mode 2 adds how far the anchor score may move before k_max changes. */
 static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid, double a,
                           double *margin)
 {
@@ -323,17 +339,18 @@ static int row_keep_count(const spo_params *pr, const ranked *r, int n_mid, doub
     }
     if (m > k_max) {
         /* the cap binds: the set is the top k_max; it would change only if
-         * the rank order at the cut changed or the mass at k_max reached p */
+         * the rank order at the cut changed or p fell to the mass of the
+         * k_max - 1 best blocks */
         double cum = 0.0;
-        for (int i = 0; i < k_max; ++i)
+        for (int i = 0; i + 1 < k_max; ++i)
             cum += exp(r[i].s - mx) / z;
-        double mg = pr->top_p - cum;
+        double mg = k_max >= 2 ? pr->top_p - cum : INFINITY;
         if (k_max > 0 && k_max < n_mid && r[k_max - 1].s - r[k_max].s < mg)
             mg = r[k_max - 1].s - r[k_max].s;
         *margin = mg < margin_k ? mg : margin_k;
         return k_max;
     }
-    double mg = pr->top_p - c_prev;
+    double mg = m >= 2 ? pr->top_p - c_prev : INFINITY;
     if (m < n_mid && c - pr->top_p < mg && m < k_max)
         mg = c - pr->top_p;
     if (m < n_mid && r[m - 1].s - r[m].s < mg)
