@@ -94,6 +94,8 @@ def lib():
         L.spo_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         L.spo_e4m3_to_f64.restype = ctypes.c_double
         L.spo_num_threads.restype = ctypes.c_int
+        L.spo_set_num_threads.argtypes = [ctypes.c_int]
+        L.spo_set_num_threads.restype = None
         L.spo_round_bf16.argtypes = [ctypes.c_double]
         L.spo_round_bf16.restype = ctypes.c_double
         L.spo_round_bf16_array.argtypes = [P, ctypes.c_int64]
@@ -112,6 +114,11 @@ def _c(a, dtype):
 
 def num_threads() -> int:
     return lib().spo_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the following calls (timing of a one-core run)."""
+    lib().spo_set_num_threads(n)
 
 
 def bf16_to_f64(bits: int) -> float:

@@ -1,4 +1,11 @@
-"""Hand workload tensors to the float64 oracle as the exact stored bytes."""
+"""Hand workload tensors to the float64 oracle as the exact stored bytes.
+
+Marshalling only (bit patterns, sizes, parameters, one request's pages
+gathered in logical order); none of the method's arithmetic.  Like the rest
+of this package it is test infrastructure: the tests, the smoke check and the
+benchmark's CPU-baseline and reference legs use it; the CUDA library never
+does.
+"""
 from __future__ import annotations
 
 import numpy as np
@@ -63,3 +70,26 @@ def run_oracle(inp: dict, params=None, units=None, max_sel=None) -> dict:
     return oracle.decode(dims_of(inp, max_sel), params or params_of(w), a["q"], a["k_cache"],
                          a["v_cache"], a["k_scale"], a["v_scale"], a["block_table"],
                          a["seq_lens"], units=units)
+
+
+def subproblem(inp: dict, b: int) -> dict:
+    """Request b alone, its pages gathered in logical order (page id = block id)."""
+    w = inp["workload"]
+    L = int(inp["seq_lens"][b])
+    P = w.block_size
+    nb = max(1, (L + P - 1) // P)
+    pages = inp["block_table"][b, :nb].long().clamp_min(0)
+    sub = dict(inp)
+    sub["workload"] = w.replace(batch=1)
+    sub["q"] = inp["q"][b:b + 1]
+    sub["k_cache"] = inp["k_cache"][pages].contiguous()
+    sub["v_cache"] = inp["v_cache"][pages].contiguous()
+    sub["k_scale"] = inp["k_scale"][pages].contiguous()
+    sub["v_scale"] = inp["v_scale"][pages].contiguous()
+    bt = torch.full((1, inp["max_blocks"]), -1, dtype=torch.int32, device=inp["q"].device)
+    bt[0, :nb] = torch.arange(nb, dtype=torch.int32, device=bt.device)
+    sub["block_table"] = bt
+    sub["seq_lens"] = inp["seq_lens"][b:b + 1]
+    sub["num_pages"] = nb
+    sub["page_of_block"] = pages
+    return sub

@@ -615,3 +615,14 @@ int spo_num_threads(void)
     return 1;
 #endif
 }
+
+/* Set the number of OpenMP threads later calls use (no effect without
+ * OpenMP); the timing of a one-core run of the oracle uses it. */
+void spo_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -20,7 +20,7 @@ import torch
 import oracle
 from block_sparse_kv_spattn_b200.workloads import make_inputs
 from cases import SMALL_ANCHOR
-from oracle_io import dequant, run_oracle
+from oracle.marshal import dequant, run_oracle
 from test_oracle_pins import _brute_topp, _select_rows
 
 pytestmark = pytest.mark.filterwarnings("ignore")

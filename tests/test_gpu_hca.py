@@ -21,7 +21,7 @@ import oracle
 from block_sparse_kv_spattn_b200 import spattn
 from block_sparse_kv_spattn_b200.workloads import WORKLOADS, Workload, make_inputs
 from tests.cases import CHUNK2_TOPP, CHUNK16_FP8, GQA8_TOPP, MQA16_TOPK, SMALL_FP8_CHUNK, SMALL_RAGGED, SMALL_TOPP
-from tests.oracle_io import dims_of, host_arrays, params_of
+from oracle.marshal import dims_of, host_arrays, params_of
 from tests.parity import OUT_TOL, lib_params, run_library
 
 pytestmark = pytest.mark.gpu

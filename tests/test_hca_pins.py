@@ -20,7 +20,7 @@ import torch
 import oracle
 from block_sparse_kv_spattn_b200.workloads import make_inputs
 from cases import SMALL_FP8_CHUNK, SMALL_TOPP
-from oracle_io import dequant, dims_of, host_arrays, params_of
+from oracle.marshal import dequant, dims_of, host_arrays, params_of
 
 GROUP = 2   # blocks per pooled entry (128 tokens)
 

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 from block_sparse_kv_spattn_b200.workloads import WORKLOADS, Workload, make_inputs
-from tests.oracle_io import bits16, dequant, dims_of, host_arrays, params_of, run_oracle
+from oracle.marshal import bits16, dequant, dims_of, host_arrays, params_of, run_oracle
 
 from tests.cases import SMALL_FP8_CHUNK, SMALL_RAGGED, SMALL_TOPP
 
