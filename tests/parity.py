@@ -22,7 +22,7 @@ import torch
 
 import oracle
 from block_sparse_kv_spattn_b200 import spattn
-from tests.oracle_io import bits16, cache_bytes, dims_of, params_of
+from oracle.marshal import bits16, cache_bytes, dims_of, params_of, subproblem
 
 MARGIN = 1e-4
 TOPP_BAND = 1e-5
@@ -61,29 +61,6 @@ def run_library(inp: dict, params: spattn.Params | None = None, kbar_bf16: bool 
                 status=status, max_sel=max_sel)
 
 
-def subproblem(inp: dict, b: int) -> dict:
-    """Request b alone, its pages gathered in logical order (page id = block id)."""
-    w = inp["workload"]
-    L = int(inp["seq_lens"][b])
-    P = w.block_size
-    nb = max(1, (L + P - 1) // P)
-    pages = inp["block_table"][b, :nb].long().clamp_min(0)
-    sub = dict(inp)
-    sub["workload"] = w.replace(batch=1)
-    sub["q"] = inp["q"][b:b + 1]
-    sub["k_cache"] = inp["k_cache"][pages].contiguous()
-    sub["v_cache"] = inp["v_cache"][pages].contiguous()
-    sub["k_scale"] = inp["k_scale"][pages].contiguous()
-    sub["v_scale"] = inp["v_scale"][pages].contiguous()
-    bt = torch.full((1, inp["max_blocks"]), -1, dtype=torch.int32, device=inp["q"].device)
-    bt[0, :nb] = torch.arange(nb, dtype=torch.int32, device=bt.device)
-    sub["block_table"] = bt
-    sub["seq_lens"] = inp["seq_lens"][b:b + 1]
-    sub["num_pages"] = nb
-    sub["page_of_block"] = pages
-    return sub
-
-
 def anchor_cap(w, row_scores: np.ndarray, S: int, nb: int) -> int:
     """The anchor-adaptive cap of one score row, computed as the library does
     (double arithmetic on the fp32 scores and parameters)."""
@@ -118,13 +95,16 @@ def _topp_prefix_ok(w, row_scores: np.ndarray, S: int, nb: int, got_mid: list[in
     return bool(near) and min(near) < TOPP_BAND
 
 
-def compare(inp: dict, gpu: dict, requests=None, params_override=None, kbar_bf16: bool = False) -> dict:
-    """Compare every step for the listed requests (default: all).  Returns a
-    summary (max errors, exact/replayed row counts); raises AssertionError on
-    any violation."""
+def compare(inp: dict, gpu: dict, requests=None, params_override=None, kbar_bf16: bool = False,
+            attend_requests=None) -> dict:
+    """Compare every step for the listed requests (default: all); the
+    attention only for ``attend_requests`` (default: the same requests).
+    Returns a summary (max errors, exact/replayed row counts); raises
+    AssertionError on any violation."""
     w = inp["workload"]
     fp8 = w.kv_fp8
     requests = range(w.batch) if requests is None else requests
+    attend_requests = set(requests if attend_requests is None else attend_requests)
     summary = dict(kbar_err=0.0, score_err=0.0, out_err=0.0, exact_rows=0, replayed_rows=0)
     assert gpu["status"] == 0, f"device status word {gpu['status']:#x}"
     opar = params_of(w, **(params_override or {}))
@@ -187,6 +167,9 @@ def compare(inp: dict, gpu: dict, requests=None, params_override=None, kbar_bf16
                         f"replay b={b} h={h}: not a valid top-p cut"
                 summary["replayed_rows"] += 1
         # 4. attention over the GPU's own selection
+        if b not in attend_requests:
+            continue
+        summary["attended"] = summary.get("attended", 0) + 1
         sel_g = np.full((1, H, gpu["max_sel"]), -1, np.int32)
         sel_g[0] = g_idx
         out_o = oracle.attend(dims, opar, qh, kh, vh, ksc, vsc, bt, sl, sel_g, g_cnt[None])

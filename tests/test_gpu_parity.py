@@ -40,8 +40,25 @@ FULL = {
 }
 
 
+# Least number of (request, KV head) rows whose selection must be decided
+# bit-exactly (oracle margin > 1e-4) at full size.  Where the cut falls among
+# noise blocks the rank gap there is often below 1e-4 and the row is checked
+# by replay instead; the floors are set well under the measured counts so
+# that a margin that collapsed to zero (every row replayed) fails.
+EXACT_FLOOR = {
+    "tiny_4k_gqa4": 2,            # of 2: the cut sits among well separated noise scores
+    "decode_128k_b8": 16,         # of 64
+    "ragged_b32": 110,            # of 256
+    "decode_1m_mqa": 0,           # of 2: the cut falls inside ~15K noise scores
+    "chunk16_fp8_512k": 0,        # of 32: a row is the minimum over its 16 tokens' cuts
+    "decode_128k_b8_anchor": 12,  # of 64
+}
+
+
 @pytest.mark.parametrize("name", list(FULL), ids=list(FULL))
 def test_full_size_sampled_parity(name):
+    """Compressed keys, scores and selection of every request; attention of
+    the sampled requests."""
     w = WORKLOADS[name]
     inp = make_inputs(w, device="cuda")
     gpu = run_library(inp)
@@ -49,11 +66,13 @@ def test_full_size_sampled_parity(name):
     if reqs is None:
         sl = inp["seq_lens"].cpu()
         reqs = [int(sl.argmin()), int(sl.argmax())]
-    s = compare(inp, gpu, requests=reqs)
+    s = compare(inp, gpu, attend_requests=reqs)
     assert s["out_err"] <= (2e-2 if w.kv_fp8 else 2e-3)
-    # every request's counts obey the rule, sampled or not
-    cnt = gpu["sel_count"].cpu().numpy()
-    assert cnt.max() <= gpu["max_sel"]
+    assert s["attended"] == len(set(reqs))
+    rows = w.batch * w.num_kv_heads
+    print(f"{name}: selection rows exact {s['exact_rows']} replayed {s['replayed_rows']} of {rows}")
+    assert s["exact_rows"] + s["replayed_rows"] == rows
+    assert s["exact_rows"] >= EXACT_FLOOR[name]
 
 
 def test_needles_are_recalled_at_1m():
@@ -137,9 +156,8 @@ def test_bad_page_sets_status_without_fault():
 
 def test_decode_selected_with_given_selection():
     """spattn_decode_selected over a hand-given (unsorted) selection."""
-    from tests.parity import subproblem  # noqa: F401  (same helpers)
     import oracle
-    from tests.oracle_io import bits16, cache_bytes, dims_of, params_of
+    from oracle.marshal import bits16, cache_bytes, dims_of, params_of
     w = WORKLOADS["tiny_4k_gqa4"]
     inp = make_inputs(w, device="cuda")
     sel = torch.tensor([[[63, 0, 17, 5, 62, 40]] * 2], dtype=torch.int32, device="cuda")
