@@ -33,23 +33,22 @@ struct AttnArgs {
     const int32_t *sel_count;   // [B*Hkv]
     float *part_o;              // [(C + units) * records per slot][rows][D]
     float *part_ml;             // [(C + units) * records per slot][rows][2]
+    // rows: query rows per unit (Tq * group, at most 64 for attn_tcw_kernel);
+    // a (request, KV head) with more query rows is split into ntiles units
+    // of 64 rows, unit u = (b * hkv + h) * ntiles + tile, each over the same
+    // kept blocks (the query-tile outer loop of flash attention)
     int tq, hq, hkv, group, rows, units, num_pages, max_blocks, max_sel;
+    int ntiles, rows_total;     // row tiles per (request, KV head); Tq * group
     float qscale;               // sm_scale * log2(e)
-    // merge inside the attention kernel (attn_tc_kernel only): the last warp
-    // to finish a unit's tiles merges its records at the end of its CTA
-    int fuse;
-    int32_t *arrive;            // [units] tiles-per-warp arrivals, zero between calls
-    float *out;                 // [B][Tq][Hq][D]
-    float *lse;                 // nullable: [B][Tq][Hq]
 };
 
 struct StageMeta {
     int j;        // logical block id
     int page;     // page id, -1 when the block or its page is invalid
-    int unit;     // b * Hkv + h
+    int unit;     // (b * Hkv + h) * ntiles + row tile
     int flags;    // kFirst | kLast | kEnd
     int seg;      // segment id within the CTA (tensor-core kernel)
-    int pre;      // first index of the unit in the concatenated kept lists
+    int unused1;
     int qslot;    // query slot holding the segment's query rows
     int pad;
 };
@@ -58,7 +57,7 @@ constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 __host__ __device__ constexpr int align16(int x) { return (x + 15) / 16 * 16; }
 
 __device__ __forceinline__ int unit_count(const AttnArgs &a, int u) {
-    return min(max(a.sel_count[u], 0), a.max_sel);
+    return min(max(a.sel_count[a.ntiles == 1 ? u : u / a.ntiles], 0), a.max_sel);
 }
 
 // CTA whose range [c*W/C, (c+1)*W/C) holds flattened index x (0 <= x < W).

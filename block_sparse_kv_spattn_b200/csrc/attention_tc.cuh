@@ -52,7 +52,6 @@
 #pragma once
 
 #include "attention.cuh"
-#include "merge.cuh"
 #include "tcgen05.cuh"
 
 namespace spattn {
@@ -65,7 +64,6 @@ constexpr int kJoint = 8;                      // StageMeta flag: S of this odd 
 constexpr int kTcWarpSlots = 4;                // partial records per (CTA, unit)
 constexpr int kTcTmemCols = 512;               // S: 4 x NQ | O: 2 x 128
 constexpr float kTcSlack = 16.f;               // log2 headroom above the reference
-constexpr int kTcMaxPend = 8;                  // units a softmax warp may hold for the merge at its CTA's end
 
 // Shared-memory layout for RQ processed query rows.  Query slots first (a
 // product with N = 16 reads rows 8-15 past a slot of 8 rows; those columns
@@ -148,8 +146,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     using TL = TcLayout<RQ>;
     constexpr int kStages = TL::kStages;
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ int4 s_pend[4][kTcMaxPend];       // (unit, first index, kept count) merged at the end
-    __shared__ int s_npend[4];
     uint8_t *pbuf = smem + TL::kOffP;
     uint8_t *qslots = smem + TL::kOffQ;
     StageMeta *meta = reinterpret_cast<StageMeta *>(smem + TL::kOffMeta);
@@ -210,7 +206,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int64_t lo = W * c / C, hi = W * (c + 1) / C;
         int i_push = 0, seg = -1, qs = 0;   // seg: current segment id, qs: its query slot
         int prev_seg = -1, prev_page = -1;  // the tile pushed last
-        int upre = 0;                       // the pushed unit's first index in the kept lists
         constexpr int kQTasks = TL::kQRows * 16 / 32;
         uint4 qreg[kQTasks];                // this lane's share of the next segment's query rows
         // Push one stage (whole warp, uniformly): wait for the stage, write the
@@ -240,7 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // loaded: one S product for the two
             const bool joint = (i_push & 1) && !(flags & kEnd) && page >= 0 && prev_page >= 0 && prev_seg == seg;
             if (lane == 0) {
-                meta[s] = StageMeta{j, page, unit, flags | (joint ? kJoint : 0), seg, upre, qs, 0};
+                meta[s] = StageMeta{j, page, unit, flags | (joint ? kJoint : 0), seg, 0, qs, 0};
                 if (page >= 0) {
                     const int y = (page * a.hkv + unit % a.hkv) * kBlock;
                     mbar_arrive_expect_tx(&full[s], kTcStageBytes);
@@ -276,7 +271,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int ia = (int)(lo > us ? lo - us : 0);
                 const int ib = (int)(hi - us < uc ? hi - us : uc);
                 const int32_t *sel = a.sel_idx + (int64_t)unit * a.max_sel;
-                upre = (int)us;   // below 2^31 whenever the kernel merges (host check)
                 // the segment's query rows (bf16 as stored, zero padded), into registers now
 #pragma unroll
                 for (int e = 0; e < kQTasks; ++e) {
@@ -453,15 +447,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float m_ref[RQ], l_run[RQ];
     int cur_seg = -1, unit = 0, L = 0, k_last = -1;
     bool had_pv = false;   // a PV product of this segment has written this warp's lanes
-    // merge in this kernel: the segment's unit (first index, kept count), the
-    // stages this warp saw of it, the units this warp will merge at the end,
-    // and the length W of the concatenated kept lists
-    int seg_pre = 0, seg_cnt = 0, n_seen = 0, n_pend = 0;
-    int64_t W_all = 0;
-    if (a.fuse) {
-        for (int u = lane; u < a.units; u += 32) W_all += unit_count(a, u);
-        for (int o = 16; o > 0; o >>= 1) W_all += __shfl_xor_sync(0xffffffffu, W_all, o);
-    }
 
     for (int k = 0;; ++k) {
         const int i = 2 * k + pr, s = i % kStages;
@@ -505,30 +490,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             tc_fence_before();
             cur_seg = -1;
-            if (a.fuse) {
-                // the record is out: count this warp's stages of the unit.
-                // Each tile is seen by both warps of its pair, so the warp
-                // whose count completes 2 x cnt is the unit's last; it merges
-                // the unit's rows at the end of this CTA and clears the count
-                // for the next call.
-                __threadfence();
-                __syncwarp();
-                int last = 0;
-                if (lane == 0) {
-                    last = atomicAdd(a.arrive + unit, n_seen) + n_seen == 2 * seg_cnt;
-                    if (last) a.arrive[unit] = 0;
-                }
-                if (__shfl_sync(0xffffffffu, last, 0)) {
-                    if (n_pend < kTcMaxPend) {
-                        if (lane == 0) s_pend[warp][n_pend] = make_int4(unit, seg_pre, seg_cnt, 0);
-                        ++n_pend;
-                    } else {
-                        __threadfence();
-                        for (int r = 0; r < a.rows; ++r)
-                            tc_merge_row(a, unit, r, seg_pre, seg_cnt, W_all, C, kTcWarpSlots);
-                    }
-                }
-            }
         }
         if (end) break;
         if (cur_seg < 0) {
@@ -537,16 +498,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             L = a.seq_lens[unit / a.hkv];
             L = (L < 0 || L > a.max_blocks * kBlock) ? 0 : L;
             had_pv = false;
-            seg_pre = md.pre;
-            seg_cnt = a.fuse ? unit_count(a, unit) : 0;
-            n_seen = 0;
 #pragma unroll
             for (int r = 0; r < RQ; ++r) {
                 m_ref[r] = -INFINITY;
                 l_run[r] = 0.f;
             }
         }
-        ++n_seen;
         const bool valid = md.page >= 0;
         const int pos = md.j * kBlock + tok;
         // ---- scores of this lane's token, in log2 units, masked
@@ -634,23 +591,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(done);
-    if (a.fuse) {
-        // ---- the units whose last arrival was in this CTA, one (unit, row)
-        // per warp at a time; then the rows of units with nothing kept
-        // (unit u by CTA u mod C)
-        if (lane == 0) s_npend[warp] = n_pend;
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // the four softmax warps
-        __threadfence();
-        const int np = s_npend[0] + s_npend[1] + s_npend[2] + s_npend[3];
-        for (int job = warp; job < np * a.rows; job += 4) {
-            int x = job / a.rows, w = 0;
-            while (w < 3 && x >= s_npend[w]) x -= s_npend[w++];
-            const int4 e = s_pend[w][x];
-            tc_merge_row(a, e.x, job % a.rows, e.y, e.z, W_all, C, kTcWarpSlots);
-        }
-        for (int u = c + C * warp; u < a.units; u += 4 * C)
-            if (unit_count(a, u) == 0) tc_zero_rows(a, u);
-    }
 }
 
 }  // namespace spattn

@@ -74,26 +74,33 @@ struct TcwMeta {
     int pad[3];
 };
 
-// Shared memory: two query slots (64 rows x 128 bf16 as two 64-column halves),
-// two P buffers (128 rows x 64 bf16), per stage the K and V operands (two
-// 64 x 64 bf16 boxes each) and, for fp8, the staging of the copied codes;
-// then meta and barriers.  Operand tiles on 1024-byte boundaries.  (A
-// separate, deeper staging ring released at conversion measured slower: the
-// converters then wait on the products instead of on the copies.)
+// Shared memory: two query slots (64 rows x 128 bf16 as two 64-column halves,
+// or the two e4m3 terms of the rows), two P buffers (128 rows x 64 bf16 or
+// f16), the copy stages and operands below, then meta and barriers.  Operand
+// tiles on 1024-byte boundaries.
+//
+// bf16 caches: kSrc = kOp stages, each the K and V operands of one block
+// (copied straight into the operand layout), released when the block's PV
+// product is done.
+// fp8 caches: a ring of kSrc copy stages, each [K codes 8 KB | V codes 8
+// KB] of one block (the K codes are the QK operand as copied), released once
+// the block's QK product is done and its V codes are converted; and kOp = 2
+// buffers of converted V (f16 operand), released by the PV product.  A copy
+// stage therefore lives for the copy, QK and the conversion only, so that
+// many blocks' copies are in flight.  Meta entries outlive the stage (the PV
+// product reads them last): kMeta = kSrc + 8, see the producer.
 template <bool FP8>
 struct TcwLayout {
-    static constexpr int kOp = FP8 ? 3 : 4;          // stages (bf16 K and V operands of a block)
-    static constexpr int kStg = FP8 ? kOp : 0;       // fp8: the staging buffer of each stage
-    static constexpr int kSrc = kOp;                 // the ring the copies land in
-    static constexpr int kMeta = kOp;                // tiles in flight at most
+    static constexpr int kOp = FP8 ? 2 : 4;          // bf16: stages; fp8: converted V buffers
+    static constexpr int kSrc = FP8 ? 7 : kOp;       // the ring the copies land in
+    static constexpr int kMeta = FP8 ? kSrc + 8 : kOp;
     static constexpr int kQSlot = kTcwRows * 256;
     static constexpr int kOffQ = 0;
     static constexpr int kOffP = kOffQ + 2 * kQSlot;                   // [2] P buffers
-    static constexpr int kOffK = kOffP + 2 * 128 * 128;
-    static constexpr int kOffV = kOffK + kOp * 16384;
-    static constexpr int kOffStg = kOffV + kOp * 16384;                // fp8: [stage][K | V] codes
-    static constexpr int kOffMeta = kOffStg + kStg * 16384;
-    static constexpr int kNBars = 3 * kOp + 5 * 2 + 2;
+    static constexpr int kOffK = kOffP + 2 * 128 * 128;                // bf16: K operands; fp8: the copy ring
+    static constexpr int kOffV = kOffK + kSrc * 16384;                 // V operands
+    static constexpr int kOffMeta = kOffV + kOp * 16384;
+    static constexpr int kNBars = 2 * kSrc + kOp + 6 * 2 + 2;
     static constexpr int kOffBars = align16(kOffMeta + kMeta * (int)sizeof(TcwMeta));
     static constexpr int kSmem = align16(kOffBars + kNBars * 8 + 16);
 };
@@ -109,6 +116,45 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes) {
     const uint32_t mag = (h2 >> 3) & 0x0fff0fffu;               // 0, or >= 0x300 (2^-9) per half
     const uint32_t nz = ((mag + 0x0d000d00u) & 0x10001000u) >> 12;   // 1 per nonzero half
     return (nz * 0x3800u + mag) | (h2 & 0x80008000u);
+}
+
+// Two e4m3 codes (low byte first) -> two f16 (low half first): one hardware
+// conversion, exact (every e4m3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(codes & 0xffffu)));
+    return h2;
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B, fp32 accumulator.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem], 8-bit operands (32 elements of K per product).
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Two floats -> two e4m3 codes (x0 in the low byte), round to nearest even,
+// saturating at +-448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float x0, float x1) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+    return r;
+}
+
+// f16 instruction descriptor (kind::f16 with f16 A and B), fp32 accumulator.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
 }
 
 // 2^x by the hardware approximation (relative error ~2^-22), results below
@@ -149,39 +195,47 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
     attn_tcw_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, AttnArgs a) {
     using TL = TcwLayout<FP8>;
     constexpr int kOp = TL::kOp, kSrc = TL::kSrc, kMeta = TL::kMeta;
+    static_assert(!FP8 || kOp == 2, "fp8: V buffer of tile k is k & 1, the PV buffers' index");
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *pbuf = smem + TL::kOffP;
     TcwMeta *meta = reinterpret_cast<TcwMeta *>(smem + TL::kOffMeta);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TL::kOffBars);
-    uint64_t *full = bars;                      // [kOp] copies landed
-    uint64_t *conv = full + kSrc;               // [kOp] operands ready (converters)
-    uint64_t *empty = conv + kOp;               // [kOp] products done with the operand stage
+    uint64_t *full = bars;                      // [kSrc] copies landed
+    uint64_t *empty = full + kSrc;              // [kSrc] the copy stage may be refilled
+    uint64_t *conv = empty + kSrc;              // [kOp] bf16: stage's operands ready; fp8: V buffer converted
     // per-buffer barriers ([k & 1] for tile k), so that no parity wait can
     // be lapped by a phase two tiles ahead
-    uint64_t *s_full = empty + kOp;             // [2] S buffer computed
+    uint64_t *s_full = conv + kOp;              // [2] S buffer computed
     uint64_t *s_free = s_full + 2;              // [2] S buffer read (warps 0, 1)
     uint64_t *p_full = s_free + 2;              // [2] P buffer written, rescales done (warps 0-3)
     uint64_t *pv_done = p_full + 2;             // [2] the PV product of that buffer completed
     uint64_t *q_free = pv_done + 2;             // [2] query slot's last product completed
-    uint64_t *fin = q_free + 2;                 // MMA issuer: all products completed
+    uint64_t *q_read = q_free + 2;              // [2] fp8: the slot's row scales read (warps 0, 1)
+    uint64_t *fin = q_read + 2;                 // MMA issuer: all products completed
     uint64_t *done = fin + 1;                   // warps 0-3 finished with TMEM
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = gridDim.x, c = blockIdx.x;
-    constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 64, false, false);
-    constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 128, false, true);
+    // fp8 caches: the keys' codes straight from the copy, the query as two
+    // e4m3 terms (two products into S); bf16: one bf16 product
+    constexpr uint32_t kIdescQK = FP8 ? umma_idesc_e4m3(128, 64, false, false) : umma_idesc_bf16(128, 64, false, false);
+    __shared__ float s_qinv[2][kTcwRows];   // fp8: 2^-e of each query row's scaling
+    // fp8 caches: one f16 product (weights and values in f16); bf16: hi / lo
+    constexpr uint32_t kIdescPV = FP8 ? umma_idesc_f16(128, 128, false, true) : umma_idesc_bf16(128, 128, false, true);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kOp; ++s) {
+        for (int s = 0; s < kSrc; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&conv[s], kTcwConvWarps);
-            mbar_init(&empty[s], 1);
+            // fp8: the QK product's commit and every converter warp
+            mbar_init(&empty[s], FP8 ? 1 + kTcwConvWarps : 1);
         }
+        for (int s = 0; s < kOp; ++s) mbar_init(&conv[s], kTcwConvWarps);
         for (int p = 0; p < 2; ++p) {
             mbar_init(&s_full[p], 1);
             mbar_init(&s_free[p], 2);
             mbar_init(&q_free[p], 1);
+            mbar_init(&q_read[p], 2);
             mbar_init(&p_full[p], 2);
             mbar_init(&pv_done[p], 1);
         }
@@ -212,46 +266,94 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
         // segment start wait for the query slot and fill it, then lane 0
         // writes the stage's meta and issues the copies.
         auto push = [&](int unit, int j, int page, int flags, int nvalid) -> bool {
-            // the stage is free once its products are done
-            const int s = i_push % kOp;
+            // the stage is free once its products (bf16), or its QK product
+            // and its conversion (fp8), are done.  (fp8: refilling stage s
+            // with tile i needs the QK product of tile i - kSrc, which needs
+            // the softmax to have read the scores of tile i - kSrc - 2; by
+            // then the PV product of every tile before i - kSrc - 4 is done,
+            // so meta entry i % kMeta, kMeta = kSrc + 8, is no longer read.)
+            const int s = i_push % kSrc;
             int okw = 1;
-            if (lane == 0 && i_push >= kOp) okw = mbar_wait(&empty[s], ((i_push / kOp) - 1) & 1);
+            if (lane == 0 && i_push >= kSrc) okw = mbar_wait(&empty[s], ((i_push / kSrc) - 1) & 1);
             if (!__shfl_sync(0xffffffffu, okw, 0)) return false;
             int qs = seg & 1;
             if (flags & kFirst) {
                 ++seg;
                 qs = seg & 1;
-                if (lane == 0 && seg >= 2) okw = mbar_wait(&q_free[qs], ((seg >> 1) - 1) & 1);
+                if (lane == 0 && seg >= 2) {
+                    okw = mbar_wait(&q_free[qs], ((seg >> 1) - 1) & 1);
+                    // fp8: the softmax warps took the slot's row scales of its
+                    // previous segment (they read them at that segment's start)
+                    if (FP8 && okw) okw = mbar_wait(&q_read[qs], ((seg >> 1) - 1) & 1);
+                }
                 if (!__shfl_sync(0xffffffffu, okw, 0)) return false;
-                // the segment's query rows (bf16 as stored, zero padded)
-                const int b = unit / a.hkv, h = unit % a.hkv;
+                // the segment's query rows, zero padded: bf16 as stored, or
+                // (fp8 caches) each row scaled by 2^e (its largest element in
+                // [2^7, 2^8)) and split into two e4m3 terms q1 + q2 (exact for
+                // the elements within 2^9 of the row's largest), one 64-row
+                // panel of 128-byte rows each
+                // (row tile `tile` of the request and KV head's Tq * group rows)
+                const int un = unit / a.ntiles, tile = unit % a.ntiles;
+                const int b = un / a.hkv, h = un % a.hkv;
                 uint8_t *qd = smem + TL::kOffQ + qs * TL::kQSlot;
                 for (int task = lane; task < kTcwRows * 16; task += 32) {
-                    const int row = task >> 4, c8 = task & 15;
+                    const int row = task >> 4, c8 = task & 15;   // a half-warp holds one row
+                    const int rg = tile * kTcwRows + row;         // the row in the whole chunk
                     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (row < a.rows) {
-                        const int t = row / a.group, g = row % a.group;
+                    if (row < a.rows && rg < a.rows_total) {
+                        const int t = rg / a.group, g = rg % a.group;
                         v = *reinterpret_cast<const uint4 *>(
                             a.q + (((int64_t)b * a.tq + t) * a.hq + h * a.group + g) * kHeadDim + c8 * 8);
                     }
-                    *reinterpret_cast<uint4 *>(qd + qslot_offset(row, c8 * 8, kTcwRows)) = v;
+                    if (!FP8) {
+                        *reinterpret_cast<uint4 *>(qd + qslot_offset(row, c8 * 8, kTcwRows)) = v;
+                    } else {
+                        float f[8];
+                        bf16x8_to_f32(v, f);
+                        float mx = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
+#pragma unroll
+                        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                        // e = 7 - floor(log2 mx), kept inside the fp32 exponent range
+                        int ex = mx > 0.f ? 7 - (int)((__float_as_uint(mx) >> 23) & 0xff) + 127 : 0;
+                        ex = ex < -100 ? -100 : (ex > 100 ? 100 : ex);
+                        const float sc = __uint_as_float((uint32_t)(ex + 127) << 23);   // 2^ex
+                        uint32_t w1[4], w2[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x0 = f[2 * e] * sc, x1 = f[2 * e + 1] * sc;
+                            w1[e] = f32x2_to_e4m3x2(x0, x1);
+                            float h0, h1;   // the first term back in fp32 (exact)
+                            e4m3x2_to_f32((uint16_t)w1[e], h0, h1);
+                            w2[e] = f32x2_to_e4m3x2(x0 - h0, x1 - h1);
+                        }
+                        // 8 bytes at byte column c8 * 8 of the row (128-byte swizzle)
+                        const int off = (row >> 3) * 1024 + (row & 7) * 128 + ((((c8 >> 1) ^ row) & 7) << 4) +
+                                        (c8 & 1) * 8;
+                        *reinterpret_cast<uint2 *>(qd + off) = make_uint2(w1[0] | (w1[1] << 16), w1[2] | (w1[3] << 16));
+                        *reinterpret_cast<uint2 *>(qd + 8192 + off) =
+                            make_uint2(w2[0] | (w2[1] << 16), w2[2] | (w2[3] << 16));
+                        if (c8 == 0) s_qinv[qs][row] = __uint_as_float((uint32_t)(127 - ex) << 23);   // 2^-ex
+                    }
                 }
                 fence_proxy_async_smem();
             }
             __syncwarp();
             if (lane == 0) {
                 float ks = 1.f, vs = 1.f;
+                const int h = (unit / a.ntiles) % a.hkv;
                 if (FP8 && page >= 0) {
-                    ks = a.k_scale[(int64_t)page * a.hkv + unit % a.hkv];
-                    vs = a.v_scale[(int64_t)page * a.hkv + unit % a.hkv];
+                    ks = a.k_scale[(int64_t)page * a.hkv + h];
+                    vs = a.v_scale[(int64_t)page * a.hkv + h];
                 }
                 meta[i_push % kMeta] = TcwMeta{j, page, unit, flags, seg, nvalid, qs, ks, vs, {0, 0, 0}};
                 if (page >= 0) {
-                    const int y = (page * a.hkv + unit % a.hkv) * kBlock;
+                    const int y = (page * a.hkv + h) * kBlock;
                     if (FP8) {
                         mbar_arrive_expect_tx(&full[s], 2 * 8192);
-                        tma_load_2d(smem + TL::kOffStg + s * 16384, &kmap, 0, y, &full[s]);
-                        tma_load_2d(smem + TL::kOffStg + s * 16384 + 8192, &vmap, 0, y, &full[s]);
+                        tma_load_2d(smem + TL::kOffK + s * 16384, &kmap, 0, y, &full[s]);   // codes: the operand
+                        tma_load_2d(smem + TL::kOffK + s * 16384 + 8192, &vmap, 0, y, &full[s]);
                     } else {
                         mbar_arrive_expect_tx(&full[s], 4 * 8192);
                         tma_load_2d(smem + TL::kOffK + s * 16384, &kmap, 0, y, &full[s]);
@@ -281,10 +383,10 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                 const int64_t us = __shfl_sync(0xffffffffu, ustart, src);
                 const int uc = __shfl_sync(0xffffffffu, cnt, src);
                 const int unit = u0 + src;
-                const int b = unit / a.hkv;
+                const int b = unit / a.ntiles / a.hkv;
                 const int ia = (int)(lo > us ? lo - us : 0);
                 const int ib = (int)(hi - us < uc ? hi - us : uc);
-                const int32_t *sel = a.sel_idx + (int64_t)unit * a.max_sel;
+                const int32_t *sel = a.sel_idx + (int64_t)(unit / a.ntiles) * a.max_sel;
                 int L = a.seq_lens[b];
                 L = (L < 0 || L > a.max_blocks * kBlock) ? 0 : L;
                 const int nb = (L + kBlock - 1) / kBlock;
@@ -333,21 +435,34 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
             const int rs = i % kSrc, os = i % kOp;
             if (!mbar_wait(&full[rs], (i / kSrc) & 1)) break;
             const TcwMeta m = meta[i % kMeta];
+            if (FP8 && (m.flags & kEnd)) break;
+            // fp8: V buffer os is free once the PV product of tile i - 2 is done
+            if (FP8 && i >= 2 && !mbar_wait(&pv_done[os], ((i >> 1) - 1) & 1)) break;
             if (m.page >= 0) {
                 uint8_t *kop = smem + TL::kOffK + os * 16384, *vop = smem + TL::kOffV + os * 16384;
                 if (FP8) {
-                    const uint8_t *stg = smem + TL::kOffStg + rs * 16384;
+                    const uint8_t *stg = smem + TL::kOffK + rs * 16384;   // [K codes | V codes]
 #pragma unroll
-                    for (int e = 0; e < 1024 / (kTcwConvWarps * 32); ++e) {
-                        const int task = ct + e * kTcwConvWarps * 32;
+                    for (int e = 0; e < 512 / (kTcwConvWarps * 32); ++e) {
+                        const int task = 512 + ct + e * kTcwConvWarps * 32;   // V only (K is used as copied)
                         const bool isv = task >= 512;
                         const int tt = task & 63, c16 = (task >> 6) & 7;   // token, 16-column chunk
                         const uint4 u = *reinterpret_cast<const uint4 *>(stg + (isv ? 8192 : 0) + tt * 128 +
                                                                          ((c16 ^ (tt & 7)) << 4));
-                        uint4 w0 = make_uint4(e4m3x2_to_bf16x2(u.x), e4m3x2_to_bf16x2(u.x >> 16),
-                                              e4m3x2_to_bf16x2(u.y), e4m3x2_to_bf16x2(u.y >> 16));
-                        uint4 w1 = make_uint4(e4m3x2_to_bf16x2(u.z), e4m3x2_to_bf16x2(u.z >> 16),
-                                              e4m3x2_to_bf16x2(u.w), e4m3x2_to_bf16x2(u.w >> 16));
+                        // K to bf16 (the QK product's type); V to f16 (the PV
+                        // product takes f16 weights and values: one conversion)
+                        uint4 w0, w1;
+                        if (isv) {
+                            w0 = make_uint4(e4m3x2_to_f16x2(u.x), e4m3x2_to_f16x2(u.x >> 16),
+                                            e4m3x2_to_f16x2(u.y), e4m3x2_to_f16x2(u.y >> 16));
+                            w1 = make_uint4(e4m3x2_to_f16x2(u.z), e4m3x2_to_f16x2(u.z >> 16),
+                                            e4m3x2_to_f16x2(u.w), e4m3x2_to_f16x2(u.w >> 16));
+                        } else {
+                            w0 = make_uint4(e4m3x2_to_bf16x2(u.x), e4m3x2_to_bf16x2(u.x >> 16),
+                                            e4m3x2_to_bf16x2(u.y), e4m3x2_to_bf16x2(u.y >> 16));
+                            w1 = make_uint4(e4m3x2_to_bf16x2(u.z), e4m3x2_to_bf16x2(u.z >> 16),
+                                            e4m3x2_to_bf16x2(u.w), e4m3x2_to_bf16x2(u.w >> 16));
+                        }
                         if (isv && tt >= m.nvalid) w0 = w1 = make_uint4(0u, 0u, 0u, 0u);
                         uint8_t *box = (isv ? vop : kop) + (c16 >> 2) * 8192;
                         const int col = (c16 & 3) * 16;
@@ -364,7 +479,10 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                 fence_proxy_async_smem();
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&conv[os]);
+            if (lane == 0) {
+                mbar_arrive(&conv[os]);
+                if (FP8) mbar_arrive(&empty[rs]);   // the V codes are converted
+            }
             if (m.flags & kEnd) break;
         }
         return;
@@ -378,14 +496,15 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
             uint64_t t_idle = 0;
             while (pv < n) {
                 bool progressed = false;
-                if (pv < qk && mbar_test_wait(&p_full[pv & 1], (pv >> 1) & 1)) {   // first: a PV product frees a stage
+                if (pv < qk && mbar_test_wait(&p_full[pv & 1], (pv >> 1) & 1) &&
+                    (!FP8 || mbar_test_wait(&conv[pv & 1], (pv >> 1) & 1))) {   // first: a PV product frees a stage
                     tc_fence_after();
-                    const int s = pv % kOp;
+                    const int s = pv % kSrc;
                     const TcwMeta m = meta[pv % kMeta];
                     if (m.page >= 0) {
                         const uint32_t acc0 = last_seg == m.seg ? 1u : 0u;
                         last_seg = m.seg;
-                        const uint32_t vb = smem_u32(smem + TL::kOffV + s * 16384);
+                        const uint32_t vb = smem_u32(smem + TL::kOffV + (FP8 ? (pv & 1) : s) * 16384);
                         const uint32_t pb = smem_u32(pbuf + (pv & 1) * 16384);
                         // O hi += P rows 0-63 . V ; O lo += P rows 64-127 . V (the
                         // other 64 lanes of each product are never read)
@@ -394,39 +513,56 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                             const uint64_t bd = sw128_desc(vb + ks * 2048, 8192, 1024);
                             umma_bf16(tbase + kTcwOHi, sw128_desc(pb + ks * 32, 16, 1024), bd, kIdescPV,
                                       ks > 0 ? 1u : acc0);
-                            umma_bf16(tbase + kTcwOLo, sw128_desc(pb + 8192 + ks * 32, 16, 1024), bd, kIdescPV,
-                                      ks > 0 ? 1u : acc0);
+                            if (!FP8)
+                                umma_bf16(tbase + kTcwOLo, sw128_desc(pb + 8192 + ks * 32, 16, 1024), bd, kIdescPV,
+                                          ks > 0 ? 1u : acc0);
                         }
                         umma_commit(&pv_done[pv & 1]);
-                        umma_commit(&empty[s]);
+                        if (!FP8) umma_commit(&empty[s]);
                     } else {
                         mbar_arrive(&pv_done[pv & 1]);
-                        mbar_arrive(&empty[s]);
+                        if (!FP8) mbar_arrive(&empty[s]);
                     }
                     ++pv;
                     progressed = true;
                 }
                 if (qk < n) {
-                    const int s = qk % kOp, j = qk & 1;
-                    if (mbar_test_wait(&conv[s], (qk / kOp) & 1) &&
+                    const int s = qk % kSrc, j = qk & 1;
+                    // bf16: the stage's operands are ready; fp8: the copied K
+                    // codes are the operand (the V conversion only gates PV)
+                    if ((FP8 ? mbar_test_wait(&full[s], (qk / kSrc) & 1) : mbar_test_wait(&conv[s], (qk / kOp) & 1)) &&
                         (qk < 2 || mbar_test_wait(&s_free[j], ((qk >> 1) - 1) & 1))) {
                         const TcwMeta m = meta[qk % kMeta];
                         if (m.flags & kEnd) {
                             n = qk;
+                            if (FP8) mbar_arrive(&s_full[j]);   // the softmax warps learn the end here
                         } else {
                             tc_fence_after();
                             if (m.page >= 0) {
                                 const uint32_t qb = smem_u32(smem + TL::kOffQ + m.qslot * TL::kQSlot);
                                 const uint32_t kb = smem_u32(smem + TL::kOffK + s * 16384);
+                                if (FP8) {
+                                    // S = q1 . K + q2 . K, 32 elements of d per product
 #pragma unroll
-                                for (int ks = 0; ks < 8; ++ks) {
-                                    const uint64_t ad = sw128_desc(qb + (ks >> 2) * (kTcwRows * 128) + (ks & 3) * 32, 16, 1024);
-                                    const uint64_t bd = sw128_desc(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                                    umma_bf16(tbase + j * 64, ad, bd, kIdescQK, ks > 0);
+                                    for (int ks = 0; ks < 8; ++ks) {
+                                        const uint64_t ad = sw128_desc(qb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                                        const uint64_t bd = sw128_desc(kb + (ks & 3) * 32, 16, 1024);
+                                        umma_f8(tbase + j * 64, ad, bd, kIdescQK, ks > 0);
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int ks = 0; ks < 8; ++ks) {
+                                        const uint64_t ad =
+                                            sw128_desc(qb + (ks >> 2) * (kTcwRows * 128) + (ks & 3) * 32, 16, 1024);
+                                        const uint64_t bd = sw128_desc(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                                        umma_bf16(tbase + j * 64, ad, bd, kIdescQK, ks > 0);
+                                    }
                                 }
                                 umma_commit(&s_full[j]);
+                                if (FP8) umma_commit(&empty[s]);   // the K codes are no longer read
                             } else {
                                 mbar_arrive(&s_full[j]);
+                                if (FP8) mbar_arrive(&empty[s]);
                             }
                             // the slot is free once the segment's last product is done
                             if (m.flags & kLast) umma_commit(&q_free[m.qslot]);
@@ -460,17 +596,19 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
     // ============================================== softmax (warps 0, 1)
     const int r = warp * 32 + lane;                       // query row (TMEM lane)
     const uint32_t lanes = (uint32_t)(warp * 32) << 16;
-    const int t_r = r / a.group;                          // the row's chunk token
-    const bool row_ok = r < a.rows;
+    int t_r = 0;             // the row's chunk token (in the current segment's row tile)
+    bool row_ok = false;     // the row exists in that tile
 
+    constexpr float kSlack = FP8 ? 15.f : kTcSlack;   // f16 weights stay below 2^15
     float m_ref = -INFINITY, l_run = 0.f;
+    float q_inv = 1.f;   // fp8: 2^-e, the scaling of this row's query in the current segment
     int cur_seg = -1, unit = 0, L = 0, k_last = -1;
     bool had_pv = false;
     // wait for tile kk's PV products (its buffer's barrier)
     auto wait_pv = [&](int kk) -> bool { return mbar_wait(&pv_done[kk & 1], (kk >> 1) & 1); };
     auto rescale_o = [&](float f) {   // both parts of this row's accumulator
 #pragma unroll 1
-        for (int cc = 0; cc < 16; ++cc) {
+        for (int cc = 0; cc < (FP8 ? 8 : 16); ++cc) {
             const uint32_t col = (cc < 8 ? kTcwOHi : kTcwOLo) + (cc & 7) * 16;
             float v[16];
             tmem_ld16(tbase + lanes + col, v);
@@ -482,8 +620,9 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
     };
 
     for (int k = 0;; ++k) {
-        // operands of tile k ready (also publishes its meta)
-        if (!mbar_wait(&conv[k % kOp], (k / kOp) & 1)) break;
+        // bf16: the operands of tile k are ready (which publishes its meta);
+        // fp8: its scores are (the MMA issuer read the meta first)
+        if (!mbar_wait(FP8 ? &s_full[k & 1] : &conv[k % kOp], FP8 ? (k >> 1) & 1 : (k / kOp) & 1)) break;
         const TcwMeta md = meta[k % kMeta];
         const bool end = md.flags & kEnd;
         if (cur_seg >= 0 && (end || md.seg != cur_seg)) {
@@ -497,9 +636,11 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                 float v[16], w[16];
                 if (had_pv) {
                     tmem_ld16(tbase + lanes + kTcwOHi + cc * 16, v);
-                    tmem_ld16(tbase + lanes + kTcwOLo + cc * 16, w);
+                    if (!FP8) {
+                        tmem_ld16(tbase + lanes + kTcwOLo + cc * 16, w);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] += w[e];
+                        for (int e = 0; e < 16; ++e) v[e] += w[e];
+                    }
                 } else {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) v[e] = 0.f;
@@ -517,16 +658,27 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
         if (cur_seg < 0) {
             cur_seg = md.seg;
             unit = md.unit;
-            L = a.seq_lens[unit / a.hkv];
+            L = a.seq_lens[unit / a.ntiles / a.hkv];
             L = (L < 0 || L > a.max_blocks * kBlock) ? 0 : L;
+            {
+                const int rg = (unit % a.ntiles) * kTcwRows + r;
+                row_ok = r < a.rows && rg < a.rows_total;
+                t_r = rg / a.group;
+            }
             had_pv = false;
             m_ref = -INFINITY;
             l_run = 0.f;
+            if (FP8) {
+                // this row's query scale for the segment; the slot may then be refilled
+                q_inv = s_qinv[md.qslot][r];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&q_read[md.qslot]);
+            }
         }
         const bool valid = md.page >= 0;
         const int j = k & 1;
         // ---- this row's 64 scores (one TMEM load), log2 units, masked
-        if (!mbar_wait(&s_full[j], (k >> 1) & 1)) break;
+        if (!FP8 && !mbar_wait(&s_full[j], (k >> 1) & 1)) break;
         tc_fence_after();
         float x[64];
         if (valid) tmem_ld64(tbase + lanes + j * 64, x);
@@ -537,7 +689,7 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
         uint32_t hw[32], lw[32];
         if (valid) {
             const int lim = min(L - 1, L - a.tq + t_r);   // last position the row sees
-            const float sc = a.qscale * md.ks;
+            const float sc = FP8 ? a.qscale * md.ks * q_inv : a.qscale * md.ks;
             const int pos0 = md.j * kBlock;
             float mx = -INFINITY;
             if (row_ok && pos0 + 63 <= lim) {   // the whole block is visible to the row
@@ -553,29 +705,38 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                     mx = fmaxf(mx, x[t]);
                 }
             }
-            if (mx > m_ref + kTcSlack || (m_ref == -INFINITY && mx != -INFINITY)) {
-                alpha = m_ref == -INFINITY ? 0.f : exp2f(m_ref - mx);
-                m_ref = mx;
+            // the weights enter P times the block's V scale, 2^(x + log2 vs - m):
+            // the reference m follows x + log2 vs, so that every weight stays
+            // below 2^slack (f16 weights for fp8 caches: below 2^15 < 65504);
+            // the row sum takes 2^(x - m), the weights divided by the scale
+            const float lvs = md.vs == 1.f ? 0.f : __log2f(md.vs);
+            const float my = mx + lvs;
+            if (my > m_ref + kSlack || (m_ref == -INFINITY && mx != -INFINITY)) {
+                alpha = m_ref == -INFINITY ? 0.f : exp2f(m_ref - my);
+                m_ref = my;
                 l_run *= alpha;
             }
-            // weights times the V scale, exp2(x - m + log2 vs), as bf16 hi / lo
-            // pairs, ready before the buffer is waited for; the row sum is
-            // taken over the scaled weights and divided by the scale once
-            const float mu = (m_ref == -INFINITY ? 0.f : m_ref) - (md.vs == 1.f ? 0.f : __log2f(md.vs));
+            const float mu = (m_ref == -INFINITY ? 0.f : m_ref) - lvs;
             float ps = 0.f;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const float p0 = ex2_ftz(x[2 * e] - mu), p1 = ex2_ftz(x[2 * e + 1] - mu);
                 ps += p0 + p1;
-                // hi = p with its low 16 bits cleared (a bf16 value), lo = the
-                // exact fp32 remainder, truncated the same way: the pair keeps
-                // ~15 significant bits, with integer ops only (the exp2 pipe
-                // stays free for the exponentials)
-                const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
-                const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
-                hw[e] = __byte_perm(b0, b1, 0x7632);
-                lw[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                if (FP8) {
+                    // one f16 weight (11 significant bits)
+                    const __half2 h = __floats2half2_rn(p0, p1);
+                    hw[e] = *reinterpret_cast<const uint32_t *>(&h);
+                } else {
+                    // hi = p with its low 16 bits cleared (a bf16 value), lo =
+                    // the exact fp32 remainder, truncated the same way: the
+                    // pair keeps ~15 significant bits, with integer ops only
+                    // (the exp2 pipe stays free for the exponentials)
+                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                    const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
+                    const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+                    hw[e] = __byte_perm(b0, b1, 0x7632);
+                    lw[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                }
             }
             l_run += md.vs == 1.f ? ps : ps / md.vs;
         }
@@ -594,8 +755,9 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
             for (int c8 = 0; c8 < 8; ++c8) {
                 *reinterpret_cast<uint4 *>(pb + sw128_offset(r, c8 * 8)) =
                     make_uint4(hw[4 * c8], hw[4 * c8 + 1], hw[4 * c8 + 2], hw[4 * c8 + 3]);
-                *reinterpret_cast<uint4 *>(pb + sw128_offset(64 + r, c8 * 8)) =
-                    make_uint4(lw[4 * c8], lw[4 * c8 + 1], lw[4 * c8 + 2], lw[4 * c8 + 3]);
+                if (!FP8)
+                    *reinterpret_cast<uint4 *>(pb + sw128_offset(64 + r, c8 * 8)) =
+                        make_uint4(lw[4 * c8], lw[4 * c8 + 1], lw[4 * c8 + 2], lw[4 * c8 + 3]);
             }
             fence_proxy_async_smem();
             had_pv = true;

@@ -26,6 +26,7 @@ struct MergeArgs {
     float *out;                 // [B][Tq][Hq][D]
     float *lse;                 // nullable: [B][Tq][Hq], ln of the row's sum of exp(logit)
     int batch, tq, hq, hkv, group, rows, units, max_sel, ctas;
+    int ntiles;                 // row tiles (units) per (request, KV head); rows = rows of one tile
     int wslots;                 // partial records per (CTA, unit): 1 (attn_tcw) or 4 (one per attn_tc softmax warp)
     int pairs;                  // 4 records: warp w's pair w / 2 took only tiles of its parity
 };
@@ -65,12 +66,13 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
     const int t = (int)((grow / a.hq) % a.tq);
     const int b = (int)(grow / ((int64_t)a.hq * a.tq));
     const int h = i / a.group, g = i % a.group;
-    const int unit = b * a.hkv + h;
-    const int row = t * a.group + g;
+    const int rg = t * a.group + g;                 // the row in the chunk's Tq * group
+    const int unit = (b * a.hkv + h) * a.ntiles + rg / a.rows;
+    const int row = rg % a.rows;
     // prefix of the unit in the concatenated sequence, and the total W
     int64_t pre = 0, W = 0;
     for (int u = lane; u < a.units; u += 32) {
-        const int cnt = min(max(a.sel_count[u], 0), a.max_sel);
+        const int cnt = min(max(a.sel_count[a.ntiles == 1 ? u : u / a.ntiles], 0), a.max_sel);
         W += cnt;
         if (u < unit) pre += cnt;
     }
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
         pre += __shfl_xor_sync(0xffffffffu, pre, o);
         W += __shfl_xor_sync(0xffffffffu, W, o);
     }
-    const int cnt = min(max(a.sel_count[unit], 0), a.max_sel);
+    const int cnt = min(max(a.sel_count[unit / a.ntiles], 0), a.max_sel);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f, M = -INFINITY;
     if (cnt > 0) {
@@ -180,112 +182,6 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     // records hold base-2 maxima of the scaled logits: ln sum = (M + log2 l) ln 2
     if (a.lse && lane == 0) a.lse[grow] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
-}
-
-
-// ------------------------------------------- merge inside the attention kernel
-
-__device__ __forceinline__ float4 ld_f4_l2(const float *p) {
-    float4 v;
-    asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ float2 ld_f2_l2(const float *p) {
-    float2 v;
-    asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
-    return v;
-}
-
-// Output row `row` (chunk token row / group, head h * group + row % group) of
-// `unit` from the unit's partial records, by one warp, as merge_kernel does
-// for one row: records of CTAs cta_of(pre) .. cta_of(pre + cnt - 1), four
-// per CTA (attn_tc_kernel's softmax warps), combined by their base-2
-// maxima.  The records were written by other CTAs of the same grid: loads go
-// to L2 (.cg), after the caller has seen every arrival.
-__device__ __forceinline__ void tc_merge_row(const AttnArgs &a, int unit, int row, int64_t pre, int cnt, int64_t W,
-                                          int C, int wslots) {
-    const int lane = threadIdx.x & 31;
-    MergeArgs m{};
-    m.ctas = C;
-    m.wslots = wslots;
-    m.pairs = wslots == 4;
-    const int c_lo = cta_of(pre, W, C), c_hi = cta_of(pre + cnt - 1, W, C);
-    const int nrec = (c_hi - c_lo + 1) * wslots;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lsum = 0.f, M = -INFINITY;
-    for (int x0 = 0; x0 < nrec; x0 += 32) {
-        const int64_t r = x0 + lane < nrec ? merge_record(m, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
-        const unsigned written = __ballot_sync(0xffffffffu, r >= 0);
-        if (!written) continue;   // uniform
-        const int64_t rfirst = __shfl_sync(0xffffffffu, r, __ffs(written) - 1);
-        const int64_t rr = r >= 0 ? r : rfirst;
-        const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
-        // rows of the first 16 records now, beside the maxima (a record that
-        // was not written reads a written one; its weight is zero)
-        float4 o16[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int64_t re = __shfl_sync(0xffffffffu, rr, e);
-            o16[e] = e < n_here ? ld_f4_l2(a.part_o + (re * a.rows + row) * kHeadDim + lane * 4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        float2 ml = make_float2(-INFINITY, 0.f);
-        if (r >= 0) ml = ld_f2_l2(a.part_ml + (r * a.rows + row) * 2);
-        const float Mb = fmaxf(M, warp_max(ml.x));
-        const unsigned valid = __ballot_sync(0xffffffffu, r >= 0 && ml.x != -INFINITY);
-        if (valid && Mb != M) {
-            const float f = M == -INFINITY ? 0.f : exp2f(M - Mb);
-            acc.x *= f;
-            acc.y *= f;
-            acc.z *= f;
-            acc.w *= f;
-            lsum *= f;
-            M = Mb;
-        }
-        float w = 0.f;
-        if ((valid >> lane) & 1u) {
-            w = exp2f(ml.x - M);
-            lsum = fmaf(w, ml.y, lsum);
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const float we = __shfl_sync(0xffffffffu, w, e);
-            acc.x = fmaf(we, o16[e].x, acc.x);
-            acc.y = fmaf(we, o16[e].y, acc.y);
-            acc.z = fmaf(we, o16[e].z, acc.z);
-            acc.w = fmaf(we, o16[e].w, acc.w);
-        }
-#pragma unroll 16
-        for (int e = 16; e < n_here; ++e) {
-            const float we = __shfl_sync(0xffffffffu, w, e);
-            const int64_t re = __shfl_sync(0xffffffffu, rr, e);
-            const float4 o = ld_f4_l2(a.part_o + (re * a.rows + row) * kHeadDim + lane * 4);
-            acc.x = fmaf(we, o.x, acc.x);
-            acc.y = fmaf(we, o.y, acc.y);
-            acc.z = fmaf(we, o.z, acc.z);
-            acc.w = fmaf(we, o.w, acc.w);
-        }
-    }
-    lsum = warp_sum(lsum);
-    const int b = unit / a.hkv, h = unit % a.hkv, t = row / a.group, g = row % a.group;
-    const int64_t grow = ((int64_t)b * a.tq + t) * a.hq + h * a.group + g;
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    reinterpret_cast<float4 *>(a.out + grow * kHeadDim)[lane] =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    if (a.lse && lane == 0) a.lse[grow] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
-}
-
-// The rows of a unit with nothing kept: zeros (log-sum-exp -inf).
-__device__ __forceinline__ void tc_zero_rows(const AttnArgs &a, int unit) {
-    const int lane = threadIdx.x & 31;
-    const int b = unit / a.hkv, h = unit % a.hkv;
-    for (int row = 0; row < a.rows; ++row) {
-        const int t = row / a.group, g = row % a.group;
-        const int64_t grow = ((int64_t)b * a.tq + t) * a.hq + h * a.group + g;
-        reinterpret_cast<float4 *>(a.out + grow * kHeadDim)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (a.lse && lane == 0) a.lse[grow] = -INFINITY;
-    }
 }
 
 }  // namespace spattn

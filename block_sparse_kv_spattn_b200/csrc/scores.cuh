@@ -19,6 +19,7 @@ struct ScoresArgs {
     const int32_t *seq_lens;
     float *scores;            // [B][Tq][Hkv][max_blocks]
     int tq, hq, num_pages, max_blocks, sink, local, bpc;
+    int tt;                   // query tokens per CTA (grid z tiles a chunk's tokens)
     int anchors;              // also score the sink and local blocks (anchor-adaptive selection)
     float scale;
 };
@@ -55,10 +56,31 @@ __device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
     return r;
 }
 
-// Grid (ceil(max_blocks / bpc), B), kScoreThreads threads.  Dynamic shared
-// memory: qbar [Tq][HKV][D] fp32, a [Tq*HKV][bpc] output tile, then the
-// page ids of the CTA's middle blocks (-1 elsewhere), read in the prologue
-// alongside the query rows.
+// Lane's 4 columns of every KV head's compressed key of one page, as fp32
+// (bf16 keys widened exactly).
+template <int HKV, bool KB16>
+__device__ __forceinline__ void load_kbar(const void *kbar, int page, int lane, float4 (&kv)[HKV]) {
+    if (KB16) {
+        const uint2 *kp =
+            reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(kbar) + (int64_t)page * HKV * kHeadDim);
+#pragma unroll
+        for (int hh = 0; hh < HKV; ++hh) {
+            const uint2 u = kp[hh * (kHeadDim / 4) + lane];
+            kv[hh] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                 __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+        }
+    } else {
+        const float4 *kp =
+            reinterpret_cast<const float4 *>(static_cast<const float *>(kbar) + (int64_t)page * HKV * kHeadDim);
+#pragma unroll
+        for (int hh = 0; hh < HKV; ++hh) kv[hh] = kp[hh * (kHeadDim / 4) + lane];
+    }
+}
+
+// Grid (ceil(max_blocks / bpc), B, ceil(Tq / tt)), kScoreThreads threads.
+// Dynamic shared memory: qbar [tt][HKV][D] fp32, a [tt*HKV][bpc] output tile,
+// then the page ids of the CTA's middle blocks (-1 elsewhere), read in the
+// prologue alongside the query rows.
 // Warp w takes blocks w, w + 4, ... of the CTA's range, BIF of them at a
 // time with all their compressed-key loads issued together.
 template <int HKV, bool KB16>
@@ -67,7 +89,9 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     constexpr int NW = kScoreThreads / 32;
     extern __shared__ float4 smem_f4[];
     float *qbar = reinterpret_cast<float *>(smem_f4);
-    const int rows = a.tq * HKV;
+    const int tb = blockIdx.z * a.tt;                 // this CTA's first query token
+    const int ntok = min(a.tt, a.tq - tb);
+    const int rows = ntok * HKV;
     float *tile = qbar + rows * kHeadDim;
     int *pages = reinterpret_cast<int *>(tile + rows * a.bpc);
     const int b = blockIdx.y;
@@ -90,7 +114,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
     for (int task = threadIdx.x; task < rows * (kHeadDim / 8); task += kScoreThreads) {
         const int c8 = task % (kHeadDim / 8), th = task / (kHeadDim / 8);
         const int hh = th % HKV, t = th / HKV;
-        const uint16_t *qr = a.q + (((int64_t)b * a.tq + t) * a.hq + hh * G) * kHeadDim + c8 * 8;
+        const uint16_t *qr = a.q + (((int64_t)b * a.tq + tb + t) * a.hq + hh * G) * kHeadDim + c8 * 8;
         float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int g0 = 0; g0 < G; g0 += 4) {  // the group's rows are loaded 4 at a time
             uint4 u[4];
@@ -142,24 +166,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
             const int jj = jb + f * NW;
             const int page = jj < a.bpc ? pages[jj] : -1;
             mid[f] = page >= 0;
-            if (mid[f]) {
-                if (KB16) {
-                    // 4 bf16 per lane: exact widening to fp32
-                    const uint2 *kp = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.kbar) +
-                                                                      (int64_t)page * HKV * kHeadDim);
-#pragma unroll
-                    for (int hh = 0; hh < HKV; ++hh) {
-                        const uint2 u = kp[hh * (kHeadDim / 4) + lane];
-                        kv[f][hh] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-                    }
-                } else {
-                    const float4 *kp = reinterpret_cast<const float4 *>(static_cast<const float *>(a.kbar) +
-                                                                        (int64_t)page * HKV * kHeadDim);
-#pragma unroll
-                    for (int hh = 0; hh < HKV; ++hh) kv[f][hh] = kp[hh * (kHeadDim / 4) + lane];
-                }
-            }
+            if (mid[f]) load_kbar<HKV, KB16>(a.kbar, page, lane, kv[f]);
         }
 #pragma unroll
         for (int f = 0; f < BIF; ++f) {
@@ -169,7 +176,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
                 for (int r = lane; r < rows; r += 32) tile[r * a.bpc + jj] = -INFINITY;
                 continue;
             }
-            for (int t0 = 0; t0 < a.tq; t0 += TPC) {
+            for (int t0 = 0; t0 < ntok; t0 += TPC) {
 #pragma unroll
                 for (int h0 = 0; h0 < HKV; h0 += HPC) {
                     float v[8];
@@ -177,7 +184,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
                     for (int i = 0; i < 8; ++i) {
                         const int tt = t0 + i / HPC, hh = h0 + i % HPC;
                         float s = 0.f;
-                        if (tt < a.tq) {
+                        if (tt < ntok) {
                             const float4 qv =
                                 reinterpret_cast<const float4 *>(qbar + (tt * HKV + hh) * kHeadDim)[lane];
                             s = qv.x * kv[f][hh].x;
@@ -191,7 +198,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
                     if ((lane & 3) == 0) {
                         const int i = lane >> 2;
                         const int tt = t0 + i / HPC, hh = h0 + i % HPC;
-                        if (tt < a.tq) tile[(tt * HKV + hh) * a.bpc + jj] = r * a.scale;
+                        if (tt < ntok) tile[(tt * HKV + hh) * a.bpc + jj] = r * a.scale;
                     }
                 }
             }
@@ -205,7 +212,7 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
         const int j = j0 + jj;
         if (j < a.max_blocks) {
             const int hh = r % HKV, t = r / HKV;
-            a.scores[(((int64_t)b * a.tq + t) * HKV + hh) * a.max_blocks + j] = tile[idx];
+            a.scores[(((int64_t)b * a.tq + tb + t) * HKV + hh) * a.max_blocks + j] = tile[idx];
         }
     }
 }

@@ -29,6 +29,7 @@ struct SelectArgs {
     float top_p, max_ratio, min_ratio;
     int n_mid_cap;             // keys capacity (>= every row's middle count)
     int sort_cap;              // power-of-two sort capacity (top-p), else 0
+    int len_early;             // the kernel before this one is the scoring grid of the same decode call
 };
 
 constexpr int kSelThreads = 1024;
@@ -294,155 +295,149 @@ __device__ void bitonic_sort_desc(unsigned long long *buf, int N) {
     }
 }
 
-// Grid (B * Hkv), block 256 / 512 / 1024 threads (longer rows, more).
-__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
-    extern __shared__ unsigned long long smem_u64[];
+// Carve the dynamic shared memory of a selection CTA.
+__device__ __forceinline__ SelectShared select_shared(const SelectArgs &a, unsigned long long *base) {
     SelectShared sh;
-    {
-        char *p = reinterpret_cast<char *>(smem_u64);
-        sh.sortbuf = reinterpret_cast<unsigned long long *>(p);
-        p += (size_t)a.sort_cap * 8;
-        sh.keys = reinterpret_cast<uint32_t *>(p);
-        p += (size_t)a.n_mid_cap * 4;
-        sh.hist = reinterpret_cast<uint32_t *>(p);
-        p += kBuckets * 4;
-        sh.cand_key = reinterpret_cast<uint32_t *>(p);
-        p += kCand * 4;
-        sh.cand_idx = reinterpret_cast<int *>(p);
-        p += kCand * 4;
-        sh.cand_ok = reinterpret_cast<int *>(p);
-        p += kCand * 4;
-        sh.itmp = reinterpret_cast<int *>(p);
-        p += 72 * 4;
-        sh.ftmp = reinterpret_cast<float *>(p);
-        p += 40 * 4;
-        sh.misc = reinterpret_cast<int *>(p);
-        p += 8 * 4;
-        sh.flags = reinterpret_cast<uint8_t *>(p);
-    }
-    const int bh = blockIdx.x;
-    const int b = bh / a.hkv, h = bh % a.hkv;
-    // When launched early behind the scoring grid of the same decode call
-    // (programmatic dependent launch), the length, which the scoring does not
-    // write, is loaded now; the scores are read only after the scoring grid
-    // completed.  Launched normally (standalone selection), the wait returns
-    // at once.
-    int L = a.seq_lens[b];
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    // the first token's score row into L1
-    {
-        const float *row0 = a.scores + ((int64_t)b * a.tq * a.hkv + h) * a.max_blocks;
-        for (int i = threadIdx.x * 32; i < a.n_mid_cap + a.sink; i += blockDim.x * 32)
-            asm volatile("prefetch.global.L1 [%0];" ::"l"(row0 + i));
-    }
+    char *p = reinterpret_cast<char *>(base);
+    sh.sortbuf = reinterpret_cast<unsigned long long *>(p);
+    p += (size_t)a.sort_cap * 8;
+    sh.keys = reinterpret_cast<uint32_t *>(p);
+    p += (size_t)a.n_mid_cap * 4;
+    sh.hist = reinterpret_cast<uint32_t *>(p);
+    p += kBuckets * 4;
+    sh.cand_key = reinterpret_cast<uint32_t *>(p);
+    p += kCand * 4;
+    sh.cand_idx = reinterpret_cast<int *>(p);
+    p += kCand * 4;
+    sh.cand_ok = reinterpret_cast<int *>(p);
+    p += kCand * 4;
+    sh.itmp = reinterpret_cast<int *>(p);
+    p += 72 * 4;
+    sh.ftmp = reinterpret_cast<float *>(p);
+    p += 40 * 4;
+    sh.misc = reinterpret_cast<int *>(p);
+    p += 8 * 4;
+    sh.flags = reinterpret_cast<uint8_t *>(p);
+    return sh;
+}
+
+// A row's length, checked (a bad one counts as empty and is reported).
+__device__ __forceinline__ int checked_len(const SelectArgs &a, int L) {
     if (L < 0 || L > a.max_blocks * kBlock) {
         if (threadIdx.x == 0) flag(SPATTN_DEV_BAD_LEN);
-        L = 0;
+        return 0;
     }
-    const int nb = (L + kBlock - 1) / kBlock;
-    const int S = a.sink, W = a.local;
-    for (int j = threadIdx.x; j < nb; j += blockDim.x) sh.flags[j] = (j < S || j >= nb - W) ? 1 : 0;
-    const int n_mid = max(0, nb - S - W);
-    // k_max = floor(ratio * n_mid), the product taken in double so that an
-    // integral product is not rounded below the integer.
-    const int k_max =
-        a.max_ratio > 0.f ? min(n_mid, (int)floor((double)a.max_ratio * (double)n_mid)) : n_mid;
-    const int k_topk = a.top_k > 0 ? min(a.top_k, k_max) : k_max;
-    __syncthreads();
+    return L;
+}
 
-    for (int t = 0; t < a.tq && n_mid > 0; ++t) {
-        const float *row = a.scores + (((int64_t)b * a.tq + t) * a.hkv + h) * a.max_blocks + S;
-        const bool anchor = a.mode == SPATTN_SEL_TOPP_ANCHOR;
-        int k = a.mode == SPATTN_SEL_TOPK ? k_topk : k_max;
-        if (k <= 0 && !anchor) continue;
-        if (a.mode == SPATTN_SEL_TOPK && k >= n_mid) {
-            for (int i = threadIdx.x; i < n_mid; i += blockDim.x) sh.flags[S + i] = 1;
+// k_max = floor(ratio * n_mid), the product taken in double so that an
+// integral product is not rounded below the integer.
+__device__ __forceinline__ int select_k_max(const SelectArgs &a, int n_mid) {
+    return a.max_ratio > 0.f ? min(n_mid, (int)floor((double)a.max_ratio * (double)n_mid)) : n_mid;
+}
+
+// The kept middle blocks of query token t of row (b, h): sh.flags[S + i] = 1
+// for each (other flags untouched).  Every thread of the CTA calls it; it
+// ends with a barrier.
+__device__ void select_token(const SelectShared &sh, const SelectArgs &a, int b, int h, int t, int nb, int n_mid) {
+    const int S = a.sink, W = a.local;
+    const int k_max = select_k_max(a, n_mid);
+    const int k_topk = a.top_k > 0 ? min(a.top_k, k_max) : k_max;
+    const float *row = a.scores + (((int64_t)b * a.tq + t) * a.hkv + h) * a.max_blocks + S;
+    const bool anchor = a.mode == SPATTN_SEL_TOPP_ANCHOR;
+    int k = a.mode == SPATTN_SEL_TOPK ? k_topk : k_max;
+    if (k <= 0 && !anchor) return;
+    if (a.mode == SPATTN_SEL_TOPK && k >= n_mid) {
+        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) sh.flags[S + i] = 1;
+        __syncthreads();
+        return;
+    }
+    uint32_t kmax_l, kmin_l, kmax, kmin;
+    load_keys(sh, row, a.n_mid_cap, &n_mid, kmax_l, kmin_l);
+    block_minmax_u32(kmax_l, kmin_l, sh.itmp, kmax, kmin);
+    if (anchor) {
+        // cap from the anchors: a = their best score, hi / lo the middle's
+        // extremes; r = clamp((hi - a) / (hi - lo), 0, 1), ratio = min_ratio
+        // + r * (max_ratio - min_ratio), k = floor(ratio * n_mid), all in
+        // double with separately rounded operations
+        const float *full = row - S;
+        float amax = -INFINITY;
+        for (int j = 0; j < S; ++j) amax = fmaxf(amax, full[j]);       // n_mid > 0: nb > S + W
+        for (int j = nb - W; j < nb; ++j) amax = fmaxf(amax, full[j]);
+        const double hi = (double)key_float(kmax), lo = (double)key_float(kmin);
+        double r = hi > lo ? __ddiv_rn(__dsub_rn(hi, (double)amax), __dsub_rn(hi, lo)) : 0.0;
+        r = r < 0.0 ? 0.0 : (r > 1.0 ? 1.0 : r);
+        const double ratio =
+            __dadd_rn((double)a.min_ratio, __dmul_rn(r, __dsub_rn((double)a.max_ratio, (double)a.min_ratio)));
+        k = min(n_mid, (int)floor(__dmul_rn(ratio, (double)n_mid)));
+        if (k <= 0) {
             __syncthreads();
-            continue;
+            return;
         }
-        uint32_t kmax_l, kmin_l, kmax, kmin;
-        load_keys(sh, row, a.n_mid_cap, &n_mid, kmax_l, kmin_l);
-        block_minmax_u32(kmax_l, kmin_l, sh.itmp, kmax, kmin);
-        if (anchor) {
-            // cap from the anchors: a = their best score, hi / lo the middle's
-            // extremes; r = clamp((hi - a) / (hi - lo), 0, 1), ratio = min_ratio
-            // + r * (max_ratio - min_ratio), k = floor(ratio * n_mid), all in
-            // double with separately rounded operations
-            const float *full = row - S;
-            float amax = -INFINITY;
-            for (int j = 0; j < S; ++j) amax = fmaxf(amax, full[j]);       // n_mid > 0: nb > S + W
-            for (int j = nb - W; j < nb; ++j) amax = fmaxf(amax, full[j]);
-            const double hi = (double)key_float(kmax), lo = (double)key_float(kmin);
-            double r = hi > lo ? __ddiv_rn(__dsub_rn(hi, (double)amax), __dsub_rn(hi, lo)) : 0.0;
-            r = r < 0.0 ? 0.0 : (r > 1.0 ? 1.0 : r);
-            const double ratio =
-                __dadd_rn((double)a.min_ratio, __dmul_rn(r, __dsub_rn((double)a.max_ratio, (double)a.min_ratio)));
-            k = min(n_mid, (int)floor(__dmul_rn(ratio, (double)n_mid)));
-            if (k <= 0) continue;
-        }
-        if (a.mode == SPATTN_SEL_TOPK) {
-            const Cut cut = find_cut(sh, n_mid, k, kmax, kmin);
+    }
+    if (a.mode == SPATTN_SEL_TOPK) {
+        const Cut cut = find_cut(sh, n_mid, k, kmax, kmin);
+        for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });
+        __syncthreads();
+        return;
+    }
+    // top-p: probabilities are the softmax of the middle scores
+    const float smax = key_float(kmax);
+    float z = 0.f;
+    for (int i = threadIdx.x; i < n_mid; i += blockDim.x) z += expf(key_float(sh.keys[i]) - smax);
+    const float Z = block_sum_f(z, sh.ftmp);
+    Cut cut{};
+    if (k < n_mid) {
+        cut = find_cut(sh, n_mid, k, kmax, kmin);
+        // mass of the k_max best blocks: below p, the cap decides alone
+        float m = 0.f;
+        for_each_in_cut(sh, n_mid, cut, [&](int i) { m += expf(key_float(sh.keys[i]) - smax); });
+        const float mass = block_sum_f(m, sh.ftmp) / Z;
+        if (mass < a.top_p) {
             for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });
             __syncthreads();
-            continue;
+            return;
         }
-        // top-p: probabilities are the softmax of the middle scores
-        const float smax = key_float(kmax);
-        float z = 0.f;
-        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) z += expf(key_float(sh.keys[i]) - smax);
-        const float Z = block_sum_f(z, sh.ftmp);
-        Cut cut{};
-        if (k < n_mid) {
-            cut = find_cut(sh, n_mid, k, kmax, kmin);
-            // mass of the k_max best blocks: below p, the cap decides alone
-            float m = 0.f;
-            for_each_in_cut(sh, n_mid, cut, [&](int i) { m += expf(key_float(sh.keys[i]) - smax); });
-            const float mass = block_sum_f(m, sh.ftmp) / Z;
-            if (mass < a.top_p) {
-                for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });
-                __syncthreads();
-                continue;
-            }
+    }
+    // the shortest prefix reaching p lies within the k candidates: sort them
+    int npow = 1;
+    while (npow < k) npow <<= 1;
+    for (int i = threadIdx.x; i < npow; i += blockDim.x) sh.sortbuf[i] = 0ull;
+    if (threadIdx.x == 0) sh.misc[4] = 0;
+    __syncthreads();
+    auto put = [&](int i) {
+        const int slot = atomicAdd(&sh.misc[4], 1);
+        sh.sortbuf[slot] = ((unsigned long long)sh.keys[i] << 32) | (0xffffffffu - (uint32_t)(S + i));
+    };
+    if (k < n_mid)
+        for_each_in_cut(sh, n_mid, cut, put);
+    else
+        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) put(i);
+    __syncthreads();
+    bitonic_sort_desc(sh.sortbuf, npow);
+    if (threadIdx.x == 0) sh.misc[5] = k;  // first crossing (default: all k)
+    __syncthreads();
+    const int per = (k + blockDim.x - 1) / blockDim.x;
+    const int lo = min(k, (int)threadIdx.x * per), hi = min(k, lo + per);
+    float local = 0.f;
+    for (int i = lo; i < hi; ++i) local += expf(key_float((uint32_t)(sh.sortbuf[i] >> 32)) - smax) / Z;
+    float c = block_incl_scan_f(local, sh.ftmp) - local;
+    for (int i = lo; i < hi; ++i) {
+        c += expf(key_float((uint32_t)(sh.sortbuf[i] >> 32)) - smax) / Z;
+        if (c >= a.top_p) {
+            atomicMin(&sh.misc[5], i + 1);
+            break;
         }
-        // the shortest prefix reaching p lies within the k candidates: sort them
-        int npow = 1;
-        while (npow < k) npow <<= 1;
-        for (int i = threadIdx.x; i < npow; i += blockDim.x) sh.sortbuf[i] = 0ull;
-        if (threadIdx.x == 0) sh.misc[4] = 0;
-        __syncthreads();
-        auto put = [&](int i) {
-            const int slot = atomicAdd(&sh.misc[4], 1);
-            sh.sortbuf[slot] = ((unsigned long long)sh.keys[i] << 32) | (0xffffffffu - (uint32_t)(S + i));
-        };
-        if (k < n_mid)
-            for_each_in_cut(sh, n_mid, cut, put);
-        else
-            for (int i = threadIdx.x; i < n_mid; i += blockDim.x) put(i);
-        __syncthreads();
-        bitonic_sort_desc(sh.sortbuf, npow);
-        if (threadIdx.x == 0) sh.misc[5] = k;  // first crossing (default: all k)
-        __syncthreads();
-        const int per = (k + blockDim.x - 1) / blockDim.x;
-        const int lo = min(k, (int)threadIdx.x * per), hi = min(k, lo + per);
-        float local = 0.f;
-        for (int i = lo; i < hi; ++i) local += expf(key_float((uint32_t)(sh.sortbuf[i] >> 32)) - smax) / Z;
-        float c = block_incl_scan_f(local, sh.ftmp) - local;
-        for (int i = lo; i < hi; ++i) {
-            c += expf(key_float((uint32_t)(sh.sortbuf[i] >> 32)) - smax) / Z;
-            if (c >= a.top_p) {
-                atomicMin(&sh.misc[5], i + 1);
-                break;
-            }
-        }
-        __syncthreads();
-        const int m = sh.misc[5];
-        for (int i = threadIdx.x; i < m; i += blockDim.x)
-            sh.flags[0xffffffffu - (uint32_t)(sh.sortbuf[i] & 0xffffffffull)] = 1;
-        __syncthreads();
     }
     __syncthreads();
+    const int m = sh.misc[5];
+    for (int i = threadIdx.x; i < m; i += blockDim.x)
+        sh.flags[0xffffffffu - (uint32_t)(sh.sortbuf[i] & 0xffffffffull)] = 1;
+    __syncthreads();
+}
 
-    // compaction: ascending block ids
+// Kept flags sh.flags[0, nb) -> ascending block ids of row bh.
+__device__ void compact_flags(const SelectShared &sh, const SelectArgs &a, int bh, int nb) {
     const int per = (nb + blockDim.x - 1) / blockDim.x;
     const int lo = min(nb, (int)threadIdx.x * per), hi = min(nb, lo + per);
     int cnt = 0;
@@ -459,6 +454,38 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         if (total > a.max_sel) flag(SPATTN_DEV_SEL_OVERFLOW);
         a.sel_count[bh] = min(total, a.max_sel);
     }
+}
+
+// Grid (B * Hkv), block 256 / 512 / 1024 threads (longer rows, more): one
+// row, its query tokens one after another, the union compacted.
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+    extern __shared__ unsigned long long smem_u64[];
+    const SelectShared sh = select_shared(a, smem_u64);
+    const int bh = blockIdx.x;
+    const int b = bh / a.hkv, h = bh % a.hkv;
+    // Launched early (programmatic dependent launch): nothing the kernel
+    // before it may write is read before the wait.  Behind the scoring grid
+    // of the same decode call (len_early), which does not write the lengths
+    // and itself started after every earlier kernel had finished, the
+    // length is loaded before the wait.
+    int L = a.len_early ? a.seq_lens[b] : 0;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!a.len_early) L = a.seq_lens[b];
+    // the first token's score row into L1
+    {
+        const float *row0 = a.scores + ((int64_t)b * a.tq * a.hkv + h) * a.max_blocks;
+        for (int i = threadIdx.x * 32; i < a.n_mid_cap + a.sink; i += blockDim.x * 32)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(row0 + i));
+    }
+    L = checked_len(a, L);
+    const int nb = (L + kBlock - 1) / kBlock;
+    const int S = a.sink, W = a.local;
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) sh.flags[j] = (j < S || j >= nb - W) ? 1 : 0;
+    const int n_mid = max(0, nb - S - W);
+    __syncthreads();
+    for (int t = 0; t < a.tq && n_mid > 0; ++t) select_token(sh, a, b, h, t, nb, n_mid);
+    __syncthreads();
+    compact_flags(sh, a, bh, nb);
 }
 
 }  // namespace spattn

@@ -61,6 +61,7 @@ spattn_status cuda_ok(cudaError_t e, const char *what) {
 // 320 SMs); the workspace is sized for it so that workspace sizes need no
 // device query.
 constexpr int kMaxAttnCtas = 2 * 160;
+constexpr int kMaxRows = 4096;   // query rows per (request, KV head): Tq * Hq / Hkv
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -84,9 +85,9 @@ spattn_status check_dims(const spattn_dims *d) {
     if (d->kbar_dtype != SPATTN_KBAR_F32 && d->kbar_dtype != SPATTN_KBAR_BF16)
         return fail(SPATTN_ERR_INVALID_ARG, "kbar_dtype %d", d->kbar_dtype);
     const int64_t rows = (int64_t)d->q_tokens * (d->num_q_heads / d->num_kv_heads);
-    if (rows > 64)
-        return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_q_heads / num_kv_heads = %lld > 64",
-                    (long long)rows);
+    if (rows > kMaxRows)
+        return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_q_heads / num_kv_heads = %lld > %d",
+                    (long long)rows, kMaxRows);
     if (d->kv_dtype != SPATTN_KV_BF16 && d->kv_dtype != SPATTN_KV_FP8_E4M3)
         return fail(SPATTN_ERR_INVALID_ARG, "kv_dtype %d", d->kv_dtype);
     if ((int64_t)d->max_blocks_per_seq * kBlock > INT32_MAX / 2)
@@ -142,6 +143,10 @@ float sm_scale_of(const spattn_params *p) {
 }
 
 int rows_of(const spattn_dims *d) { return d->q_tokens * (d->num_q_heads / d->num_kv_heads); }
+// Row tiles of (at most) 64 query rows per (request, KV head) for the
+// attention, and the rows of one tile (the stride of the partial records).
+int row_tiles(const spattn_dims *d) { return (rows_of(d) + kTcwRows - 1) / kTcwRows; }
+int tile_rows(const spattn_dims *d) { return std::min(rows_of(d), kTcwRows); }
 
 // Attention runs on the tensor cores: attn_tc_kernel for bf16 caches with
 // at most kTcNQ query rows per KV head, attn_tcw_kernel for the rest (fp8
@@ -155,17 +160,21 @@ int records_per_slot(const spattn_dims *d) { return uses_tc(d) ? kTcWarpSlots : 
 // Per-device caches (SM count; which kernels have their shared-memory limit
 // raised).  Guarded by one mutex: these are host-side set-up calls only.
 std::mutex g_mu;
-std::set<std::pair<int, const void *>> g_smem_set;
+std::map<std::pair<int, const void *>, int> g_smem_set;
 
+// Raise a kernel's dynamic shared-memory limit (per device and kernel) to
+// the largest size asked for so far, so that a call needing more than an
+// earlier one raises it again.
 spattn_status ensure_smem(const void *func, int bytes) {
     if (bytes <= 48 * 1024) return SPATTN_OK;
     int dev;
     SP_TRY(cuda_ok(cudaGetDevice(&dev), "cudaGetDevice"));
     std::lock_guard<std::mutex> lk(g_mu);
-    if (g_smem_set.count({dev, func})) return SPATTN_OK;
+    auto it = g_smem_set.find({dev, func});
+    if (it != g_smem_set.end() && it->second >= bytes) return SPATTN_OK;
     SP_TRY(cuda_ok(cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
                    "cudaFuncSetAttribute"));
-    g_smem_set.insert({dev, func});
+    g_smem_set[{dev, func}] = bytes;
     return SPATTN_OK;
 }
 
@@ -191,27 +200,19 @@ spattn_status sm_count(int *out) {
 constexpr int kMaxSmem = 227 * 1024;
 
 struct DecodeLayout {
-    size_t arrive_off, scores_off, scores_bytes, part_o_off, part_ml_off, total;
+    size_t scores_off, scores_bytes, part_o_off, part_ml_off, total;
 };
 
-// Arrival counts of the merge inside the attention kernel: a fixed region
-// at the start of every decode workspace (so that it stays in place
-// whatever the dims of the call), zero between calls.
-constexpr int kArriveUnits = 8192;
-constexpr size_t kArriveBytes = kArriveUnits * sizeof(int32_t);
-constexpr int kFuseMaxRecords = 64;   // records per unit, on average, up to which the kernel merges
-
-// Workspace: arrival counts | [scores] | partial outputs | partial (max,
-// sum).  (C_max + units) slots of `rows` query rows, records_per_slot()
-// records per slot.
+// Workspace: [scores] | partial outputs | partial (max, sum).  (C_max +
+// units) slots of `rows` query rows, records_per_slot() records per slot;
+// units count every 64-row tile of a (request, KV head) separately.  The
+// scores are there for spattn_decode without scores_out.
 DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
     DecodeLayout L{};
-    const int64_t units = (int64_t)d->batch * d->num_kv_heads;
+    const int64_t units = (int64_t)d->batch * d->num_kv_heads * row_tiles(d);
     const int64_t slots = (kMaxAttnCtas + units) * records_per_slot(d);
-    const int64_t rows = rows_of(d);
+    const int64_t rows = tile_rows(d);
     size_t off = 0;
-    L.arrive_off = 0;
-    off += align_up(kArriveBytes);
     L.scores_off = off;
     L.scores_bytes = with_scores ? align_up((size_t)d->batch * d->q_tokens * d->num_kv_heads *
                                             d->max_blocks_per_seq * sizeof(float))
@@ -279,12 +280,16 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     a.local = p->local_blocks;
     a.anchors = p->mode == SPATTN_SEL_TOPP_ANCHOR;
     a.scale = sm_scale_of(p);
-    const int rowsq = d->q_tokens * d->num_kv_heads;
-    a.bpc = score_blocks_per_cta(rowsq);
-    const int smem = rowsq * (kHeadDim + a.bpc) * (int)sizeof(float) + a.bpc * (int)sizeof(int);
-    if (smem > kMaxSmem)
+    // query tokens per CTA: at most 128 (token, KV head) rows of q-bar
+    a.tt = std::max(1, std::min(d->q_tokens, 128 / d->num_kv_heads));
+    const int rowsq = a.tt * d->num_kv_heads;
+    const int ztiles = (d->q_tokens + a.tt - 1) / a.tt;
+    const int bpc_min = score_blocks_per_cta(rowsq);   // (a one-wave grid of more blocks per CTA measured slower)
+    auto smem_of = [&](int bpc) {
+        return rowsq * (kHeadDim + bpc) * (int)sizeof(float) + bpc * (int)sizeof(int);
+    };
+    if (smem_of(bpc_min) > kMaxSmem)
         return fail(SPATTN_ERR_UNSUPPORTED, "q_tokens * num_kv_heads = %d too large for block scores", rowsq);
-    dim3 grid((d->max_blocks_per_seq + a.bpc - 1) / a.bpc, d->batch);
     const bool kb16 = d->kbar_dtype == SPATTN_KBAR_BF16;
     const void *fn = nullptr;
 #define SP_SCORES_FN(H) (kb16 ? (const void *)block_scores_kernel<H, true> : (const void *)block_scores_kernel<H, false>)
@@ -296,6 +301,9 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
         case 16: fn = SP_SCORES_FN(16); break;
     }
 #undef SP_SCORES_FN
+    a.bpc = bpc_min;
+    const int smem = smem_of(a.bpc);
+    dim3 grid((d->max_blocks_per_seq + a.bpc - 1) / a.bpc, d->batch, ztiles);
     SP_TRY(ensure_smem(fn, smem));
     cudaError_t e = cudaSuccess;
 #define SP_SCORES_LAUNCH(H)                                                                     \
@@ -312,16 +320,13 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     return cuda_ok(e, "block_scores launch");
 }
 
-// `early`: launched behind block_scores_kernel of the same call (which
-// releases its dependents at entry), so that the selection's prologue
-// overlaps the scoring.  The prologue reads seq_lens before it waits for the
-// scoring grid; that is safe only when the kernel before it in the stream is
-// that scoring grid (which does not write seq_lens, and which itself started
-// after every earlier kernel had finished).  The standalone spattn_select
-// follows whatever the caller ran last (possibly the kernel that updates
-// seq_lens), so it launches normally.
+// The selection is launched early (programmatic dependent launch): its CTAs
+// may start while the kernel before it in the stream finishes, and wait for
+// it before reading anything that kernel may write.  `behind_scores`: the
+// kernel before it is block_scores_kernel of the same decode call, so the
+// request lengths (which it does not write) may be read before the wait.
 spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const float *scores,
-                            const int32_t *sl, int32_t *sel_idx, int32_t *sel_count, bool early,
+                            const int32_t *sl, int32_t *sel_idx, int32_t *sel_count, bool behind_scores,
                             cudaStream_t st) {
     SelectArgs a;
     a.scores = scores;
@@ -340,6 +345,7 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
     a.top_p = p->top_p;
     a.max_ratio = p->max_ratio;
     a.n_mid_cap = std::max(1, n_mid_cap(d, p));
+    a.len_early = behind_scores ? 1 : 0;
     a.sort_cap = 0;
     if (p->mode != SPATTN_SEL_TOPK) {
         const int km = std::max(1, k_max_of(p, n_mid_cap(d, p)));
@@ -351,15 +357,13 @@ spattn_status launch_select(const spattn_dims *d, const spattn_params *p, const 
     if (smem > (size_t)kMaxSmem)
         return fail(SPATTN_ERR_UNSUPPORTED, "selection needs %zu bytes of shared memory (max_blocks %d)",
                     smem, a.max_blocks);
-    SP_TRY(ensure_smem((const void *)select_kernel, (int)smem));
     // latency-bound: the fewest threads that still cover a row in a few
     // passes (measured: 512 beat 1024 by 15-25 % on 2K-4K middle blocks)
     const int nm = n_mid_cap(d, p);
     const int threads = nm <= 1024 ? 256 : (nm <= 4096 ? 512 : kSelThreads);
-    const dim3 grid(d->batch * d->num_kv_heads);
-    return cuda_ok(early ? launch_early(select_kernel, grid, dim3(threads), smem, st, a)
-                         : launch(select_kernel, grid, dim3(threads), smem, st, a),
-                   "select launch");
+    const unsigned rows = (unsigned)(d->batch * d->num_kv_heads);
+    SP_TRY(ensure_smem((const void *)select_kernel, (int)smem));
+    return cuda_ok(launch_early(select_kernel, dim3(rows), dim3(threads), smem, st, a), "select launch");
 }
 
 // cuTensorMapEncodeTiled, reached through the runtime's driver entry point.
@@ -484,23 +488,15 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     a.hq = d->num_q_heads;
     a.hkv = d->num_kv_heads;
     a.group = d->num_q_heads / d->num_kv_heads;
-    a.rows = rows;
-    a.units = d->batch * d->num_kv_heads;
+    a.rows = tile_rows(d);
+    a.rows_total = rows;
+    a.ntiles = row_tiles(d);
+    a.units = d->batch * d->num_kv_heads * a.ntiles;
     a.num_pages = d->num_pages;
     a.max_blocks = d->max_blocks_per_seq;
     a.max_sel = d->max_sel;
     a.qscale = sm_scale_of(p) * kLog2e;
-    a.out = out;
-    a.lse = lse;
-    a.arrive = reinterpret_cast<int32_t *>(ws + L.arrive_off);
     const bool tc = uses_tc(d);
-    // merge inside the attention kernel when a unit's records are few (a
-    // warp merges a row at a CTA's end) and the counts fit their region
-    {
-        const int64_t recs = ((int64_t)std::min(kMaxAttnCtas, sms) / std::max(1, a.units) + 2) * kTcWarpSlots;
-        a.fuse = tc && a.units <= kArriveUnits && recs <= kFuseMaxRecords &&
-                 (int64_t)a.units * a.max_sel < ((int64_t)1 << 31);
-    }
     int ctas = 0;
     if (tc)
         SP_TRY(launch_attn_tc(a, k_cache, v_cache, sms, st, &ctas));
@@ -508,7 +504,6 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
         SP_TRY(fp8 ? launch_attn_tcw<true>(a, k_cache, v_cache, sms, st, &ctas)
                    : launch_attn_tcw<false>(a, k_cache, v_cache, sms, st, &ctas));
 
-    if (a.fuse) return SPATTN_OK;
     MergeArgs m;
     m.part_o = a.part_o;
     m.part_ml = a.part_ml;
@@ -520,8 +515,9 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.hq = d->num_q_heads;
     m.hkv = d->num_kv_heads;
     m.group = a.group;
-    m.rows = rows;
+    m.rows = a.rows;
     m.units = a.units;
+    m.ntiles = a.ntiles;
     m.max_sel = d->max_sel;
     m.ctas = ctas;
     m.wslots = records_per_slot(d);
@@ -588,7 +584,7 @@ template <bool FP8>
 constexpr bool tcw_layout_ok() {
     using TL = TcwLayout<FP8>;
     return TL::kSmem <= 227 * 1024 && TL::kOffP % 1024 == 0 && TL::kOffK % 1024 == 0 && TL::kOffV % 1024 == 0 &&
-           TL::kOffStg % 1024 == 0 && TL::kOffQ % 1024 == 0;
+           TL::kOffMeta % 16 == 0 && TL::kOffQ % 1024 == 0;
 }
 static_assert(tcw_layout_ok<false>() && tcw_layout_ok<true>(), "many-row tensor-core layout");
 
@@ -748,15 +744,6 @@ size_t spattn_decode_workspace_size(const spattn_dims *dims, const spattn_params
     return decode_layout(dims, true).total;
 }
 
-spattn_status spattn_decode_workspace_init(void *workspace, size_t workspace_bytes, spattn_stream_t stream) {
-    if (!workspace || workspace_bytes < kArriveBytes)
-        return fail(SPATTN_ERR_WORKSPACE, "workspace of %zu bytes < %zu (the arrival counts)", workspace_bytes,
-                    kArriveBytes);
-    SP_TRY(cuda_ok(cudaMemsetAsync(workspace, 0, kArriveBytes, reinterpret_cast<cudaStream_t>(stream)),
-                   "workspace init"));
-    return ok();
-}
-
 spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_params *params, const void *q,
                                      const void *k_cache, const void *v_cache, const float *k_scale,
                                      const float *v_scale, const int32_t *block_table,
@@ -811,10 +798,7 @@ spattn_status spattn_decode_selected_noalloc(const spattn_dims *dims, const spat
     void *scratch = nullptr;
     SP_TRY(noalloc_scratch(&scratch));
     char *ws = static_cast<char *>(scratch);
-    // the arrival counts must start at zero; a completed call leaves them
-    // zero, but one that gave up on a wait may not: clear them every call
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    SP_TRY(cuda_ok(cudaMemsetAsync(ws + L.arrive_off, 0, kArriveBytes, st), "clear scratch counts"));
     SP_TRY(launch_attention(dims, params, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
                             sel_idx, sel_count, out, nullptr, ws, L, st));
     return ok();

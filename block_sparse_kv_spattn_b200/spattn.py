@@ -39,7 +39,7 @@ EXPORTS = ("spattn_required_max_sel", "spattn_compress_keys", "spattn_block_scor
            "spattn_decode", "spattn_last_error", "spattn_get_device_status", "spattn_version",
            "spattn_decode_selected_noalloc", "spattn_decode_selected_lse", "spattn_hca_entries",
            "spattn_hca_pool", "spattn_hca_attend", "spattn_lse_merge", "spattn_hca_attend_merge",
-           "spattn_hca_workspace_size", "spattn_decode_workspace_init")
+           "spattn_hca_workspace_size")
 
 
 class SpattnError(RuntimeError):
@@ -110,7 +110,6 @@ def load() -> ctypes.CDLL:
         "spattn_hca_workspace_size": ([P], ctypes.c_size_t),
         "spattn_lse_merge": ([P] * 8, ctypes.c_int),
         "spattn_hca_attend_merge": ([P] * 10 + [P, ctypes.c_size_t, P], ctypes.c_int),
-        "spattn_decode_workspace_init": ([P, ctypes.c_size_t, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -168,17 +167,7 @@ def workspace_size(dims: CDims, params: Params) -> int:
 
 
 def alloc_workspace(dims: CDims, params: Params, device) -> torch.Tensor:
-    """A decode workspace, initialised (spattn_decode_workspace_init)."""
-    ws = torch.empty(workspace_size(dims, params), dtype=torch.uint8, device=device)
-    workspace_init(ws)
-    return ws
-
-
-def workspace_init(workspace: torch.Tensor, stream=None) -> None:
-    """Zero the workspace's arrival counts: once after allocation, and after
-    a call that set a device status bit."""
-    _check(load().spattn_decode_workspace_init(_p(workspace), workspace.numel() * workspace.element_size(),
-                                               _stream(stream)))
+    return torch.empty(workspace_size(dims, params), dtype=torch.uint8, device=device)
 
 
 def compress_keys(k_cache, k_scale, block_table, seq_lens, kbar, old_lens=None, *,

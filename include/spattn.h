@@ -117,7 +117,7 @@ typedef enum { SPATTN_SEL_TOPK = 0, SPATTN_SEL_TOPP = 1, SPATTN_SEL_TOPP_ANCHOR 
 typedef struct {
     int32_t batch;              /* B >= 1 */
     int32_t q_tokens;           /* Tq >= 1: query tokens per request (1 = decode) */
-    int32_t num_q_heads;        /* Hq, a multiple of Hkv; Tq * Hq / Hkv <= 64 */
+    int32_t num_q_heads;        /* Hq, a multiple of Hkv; Tq * Hq / Hkv <= 4096 */
     int32_t num_kv_heads;       /* Hkv: 1, 2, 4, 8 or 16 */
     int32_t head_dim;           /* d, must be 128 */
     int32_t block_size;         /* P, must be 64 */
@@ -204,25 +204,9 @@ spattn_status spattn_select(const spattn_dims *dims, const spattn_params *params
                             int32_t *sel_idx, int32_t *sel_count, spattn_stream_t stream);
 
 /* Bytes of workspace spattn_decode / spattn_decode_selected need (split-KV
- * partial results, per-unit arrival counts and, for spattn_decode without
- * scores_out, the scores).  Returns 0 on invalid arguments. */
+ * partial results and, for spattn_decode without scores_out, the scores).
+ * Returns 0 on invalid arguments. */
 size_t spattn_decode_workspace_size(const spattn_dims *dims, const spattn_params *params);
-
-/*
- * spattn_decode_workspace_init -- make a decode workspace ready for use.
- *
- * The attention kernel combines a unit's split partial results itself when
- * the split is shallow: the last warp to finish a unit's kept blocks (found
- * by per-unit arrival counts in the workspace) merges them.  The counts must
- * be zero when a call starts; every call that completes leaves them zero.
- * So a workspace is initialised once, after it is allocated (this call
- * zeroes the counts, asynchronously on `stream`), and again only after a
- * call that set a device status bit.  One workspace serves calls of any dims
- * that fit it; calls that may overlap on the GPU need separate workspaces.
- * Returns SPATTN_ERR_WORKSPACE when workspace is NULL or smaller than the
- * arrival count region (32 KiB).
- */
-spattn_status spattn_decode_workspace_init(void *workspace, size_t workspace_bytes, spattn_stream_t stream);
 
 /*
  * spattn_decode_selected -- exact attention over a given selection.
@@ -281,13 +265,12 @@ spattn_status spattn_decode_selected_lse(const spattn_dims *dims, const spattn_p
  * fixed scratch array built into the library (16 MiB, a module-scope device
  * array present on every GPU that loads the library until the process
  * exits).  Arguments, layouts and results are those of
- * spattn_decode_selected; dims whose scratch needs more than 16 MiB (32 KiB
- * of arrival counts, then (320 + B * Hkv) x R x (Tq * Hq / Hkv) x (d + 2) x
- * 4 bytes of partial results, R = 4 records per slot for bf16 caches with
- * Tq * Hq / Hkv <= 16, 1 otherwise) are rejected with SPATTN_ERR_UNSUPPORTED
- * before anything is enqueued.  No allocation call is made; every call
- * zeroes the arrival counts with an asynchronous memset on `stream` before
- * the attention.  The first call on each device looks up the array's device address
+ * spattn_decode_selected; dims whose partial results need more than 16 MiB
+ * ((320 + B * Hkv * T) x R x min(Tq * Hq / Hkv, 64) x (d + 2) x 4 bytes, T
+ * = the 64-row tiles of a (request, KV head), R = 4 records per slot for
+ * bf16 caches with Tq * Hq / Hkv <= 16, 1 otherwise) are rejected with
+ * SPATTN_ERR_UNSUPPORTED before anything is enqueued.  No allocation call is
+ * made.  The first call on each device looks up the array's device address
  * (a host-side CUDA runtime call), so make that first call before any stream
  * capture.  Every call on a device shares the one array and leaves its
  * contents behind; calls whose executions overlap on the GPU (different

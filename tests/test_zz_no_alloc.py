@@ -53,7 +53,7 @@ def _case(name):
 
 def test_noalloc_matches_workspace_entry_point(cuda):
     """Calls alternate between a small and a large shape (tiny, 128K, tiny,
-    128K), so a call that read partial results or counts left in the shared
+    128K), so a call that read partial results left in the shared
     scratch by the call before it would differ from the workspace entry
     point.  Both entry points run the same kernels with the same split on the
     same selection, so the outputs must be identical bit for bit."""
