@@ -53,12 +53,24 @@ namespace spattn {
 // share sub-partitions 0 and 1 only with the producer and the MMA issuer;
 // the converters (warps 2, 3, 6, 7) have sub-partitions 2 and 3 to
 // themselves.  Two warps per sub-partition leave room for 255 registers.
-constexpr int kTcwThreads = 8 * 32;
+constexpr int kTcwThreads = 8 * 32;           // bf16 caches
+constexpr int kTcwThreadsFp8 = 10 * 32;       // fp8 caches
+__host__ __device__ constexpr int tcw_threads(bool fp8) { return fp8 ? kTcwThreadsFp8 : kTcwThreads; }
 constexpr int kTcwRows = 64;                  // query rows per unit, at most
 constexpr int kTcwConvWarps = 4;
-__device__ __forceinline__ int tcw_conv_index(int warp) {   // 0..3 for a converter warp, else -1
+// Converter warps: bf16 caches 2, 3, 6, 7 (sub-partitions 2 and 3, beside the
+// two softmax warps 0 and 1); fp8 caches 6, 7, 8, 9 (the softmax warps are
+// 0-3 there).  0..3 for a converter warp, else -1.
+template <bool FP8>
+__device__ __forceinline__ int tcw_conv_index(int warp) {
+    if (FP8) return warp >= 6 && warp < 10 ? warp - 6 : -1;
     return warp == 2 ? 0 : warp == 3 ? 1 : warp == 6 ? 2 : warp == 7 ? 3 : -1;
 }
+// Softmax warps and partial records per (CTA, unit) slot: bf16 caches two
+// warps, one record; fp8 caches four warps in two halves (tokens 0-31 and
+// 32-63 of a block, each with its own reference maximum), two records.
+__host__ __device__ constexpr int tcw_softmax_warps(bool fp8) { return fp8 ? 4 : 2; }
+__host__ __device__ constexpr int tcw_records(bool fp8) { return fp8 ? 2 : 1; }
 constexpr int kTcwTmemCols = 512;             // S: 2 x 64 | O hi: 128 | O lo: 128
 constexpr int kTcwOHi = 128, kTcwOLo = 256;   // TMEM columns of the two output parts
 
@@ -92,9 +104,11 @@ struct TcwMeta {
 template <bool FP8>
 struct TcwLayout {
     static constexpr int kOp = FP8 ? 2 : 4;          // bf16: stages; fp8: converted V buffers
-    static constexpr int kSrc = FP8 ? 7 : kOp;       // the ring the copies land in
+    static constexpr int kSrc = FP8 ? 5 : kOp;       // the ring the copies land in
     static constexpr int kMeta = FP8 ? kSrc + 8 : kOp;
-    static constexpr int kQSlot = kTcwRows * 256;
+    // bf16: 64 rows x 128 bf16; fp8: the two e4m3 terms, each 128 rows (the
+    // 64 query rows twice, for the two softmax halves) x 128 bytes
+    static constexpr int kQSlot = FP8 ? 2 * 128 * 128 : kTcwRows * 256;
     static constexpr int kOffQ = 0;
     static constexpr int kOffP = kOffQ + 2 * kQSlot;                   // [2] P buffers
     static constexpr int kOffK = kOffP + 2 * 128 * 128;                // bf16: K operands; fp8: the copy ring
@@ -190,8 +204,25 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 consecutive 32-bit TMEM columns of this thread's lane, one load.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 template <bool FP8>
-__global__ void __launch_bounds__(kTcwThreads, 1)
+__global__ void __launch_bounds__(tcw_threads(FP8), 1)
     attn_tcw_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, AttnArgs a) {
     using TL = TcwLayout<FP8>;
     constexpr int kOp = TL::kOp, kSrc = TL::kSrc, kMeta = TL::kMeta;
@@ -233,19 +264,25 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
         for (int s = 0; s < kOp; ++s) mbar_init(&conv[s], kTcwConvWarps);
         for (int p = 0; p < 2; ++p) {
             mbar_init(&s_full[p], 1);
-            mbar_init(&s_free[p], 2);
+            mbar_init(&s_free[p], tcw_softmax_warps(FP8));
             mbar_init(&q_free[p], 1);
-            mbar_init(&q_read[p], 2);
-            mbar_init(&p_full[p], 2);
+            mbar_init(&q_read[p], tcw_softmax_warps(FP8));
+            mbar_init(&p_full[p], tcw_softmax_warps(FP8));
             mbar_init(&pv_done[p], 1);
         }
         mbar_init(fin, 1);
-        mbar_init(done, 2);
+        mbar_init(done, tcw_softmax_warps(FP8));
         fence_mbar_init();
     }
     if (warp == 5) {
         tmem_alloc(tmem_slot, kTcwTmemCols);
         tmem_relinquish();
+    }
+    if (FP8) {
+        // the P halves a thread never writes stay zero
+        for (int i = threadIdx.x; i < 2 * 16384 / 16; i += blockDim.x)
+            reinterpret_cast<uint4 *>(pbuf)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -331,9 +368,14 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                         // 8 bytes at byte column c8 * 8 of the row (128-byte swizzle)
                         const int off = (row >> 3) * 1024 + (row & 7) * 128 + ((((c8 >> 1) ^ row) & 7) << 4) +
                                         (c8 & 1) * 8;
-                        *reinterpret_cast<uint2 *>(qd + off) = make_uint2(w1[0] | (w1[1] << 16), w1[2] | (w1[3] << 16));
-                        *reinterpret_cast<uint2 *>(qd + 8192 + off) =
-                            make_uint2(w2[0] | (w2[1] << 16), w2[2] | (w2[3] << 16));
+                        // the row twice (rows r and 64 + r: 8 KiB apart) in each
+                        // term's 128-row panel (16 KiB apart)
+                        const uint2 t1 = make_uint2(w1[0] | (w1[1] << 16), w1[2] | (w1[3] << 16));
+                        const uint2 t2 = make_uint2(w2[0] | (w2[1] << 16), w2[2] | (w2[3] << 16));
+                        *reinterpret_cast<uint2 *>(qd + off) = t1;
+                        *reinterpret_cast<uint2 *>(qd + 8192 + off) = t1;
+                        *reinterpret_cast<uint2 *>(qd + 16384 + off) = t2;
+                        *reinterpret_cast<uint2 *>(qd + 16384 + 8192 + off) = t2;
                         if (c8 == 0) s_qinv[qs][row] = __uint_as_float((uint32_t)(127 - ex) << 23);   // 2^-ex
                     }
                 }
@@ -423,14 +465,14 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
         return;
     }
 
-    if (tcw_conv_index(warp) >= 0) {
+    if (tcw_conv_index<FP8>(warp) >= 0) {
         // ========================================================== converters
         // Stage by stage: fp8 codes -> bf16 operand boxes, V rows of unfilled
         // slots zeroed; then the operands are released to the MMA issuer.
         // Lanes take consecutive tokens of one 16-column chunk: both the
         // 128-byte-swizzled staging rows and the operand rows are then read
         // and written without bank conflicts.
-        const int ct = tcw_conv_index(warp) * 32 + lane;   // 0 .. 32 * kTcwConvWarps - 1
+        const int ct = tcw_conv_index<FP8>(warp) * 32 + lane;   // 0 .. 32 * kTcwConvWarps - 1
         for (int i = 0;; ++i) {
             const int rs = i % kSrc, os = i % kOp;
             if (!mbar_wait(&full[rs], (i / kSrc) & 1)) break;
@@ -545,7 +587,7 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                                     // S = q1 . K + q2 . K, 32 elements of d per product
 #pragma unroll
                                     for (int ks = 0; ks < 8; ++ks) {
-                                        const uint64_t ad = sw128_desc(qb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                                        const uint64_t ad = sw128_desc(qb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                                         const uint64_t bd = sw128_desc(kb + (ks & 3) * 32, 16, 1024);
                                         umma_f8(tbase + j * 64, ad, bd, kIdescQK, ks > 0);
                                     }
@@ -593,9 +635,15 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
         return;
     }
 
-    // ============================================== softmax (warps 0, 1)
-    const int r = warp * 32 + lane;                       // query row (TMEM lane)
-    const uint32_t lanes = (uint32_t)(warp * 32) << 16;
+    // ============================================== softmax (warps 0, 1; fp8: 0-3)
+    // fp8: warps 2h, 2h + 1 take tokens 32h .. 32h + 31 of every block for
+    // the 64 query rows (the query operand holds the rows twice, so TMEM lane
+    // 64h + r holds row r's scores); each half keeps its own reference
+    // maximum, sum and accumulator rows and writes its own partial record.
+    const int half = FP8 ? warp >> 1 : 0;
+    const int r = (FP8 ? (warp & 1) : warp) * 32 + lane;  // query row
+    const uint32_t lanes = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lane quarter
+    constexpr int NT = FP8 ? 32 : 64;                     // a block's tokens per thread
     int t_r = 0;             // the row's chunk token (in the current segment's row tile)
     bool row_ok = false;     // the row exists in that tile
 
@@ -629,7 +677,7 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
             // ---- end of a segment: this row's partial record (m, l, O = hi + lo)
             if (k_last >= 0 && !wait_pv(k_last)) break;
             tc_fence_after();
-            const int64_t rec = ((int64_t)c + unit) * a.rows + r;
+            const int64_t rec = (((int64_t)c + unit) * tcw_records(FP8) + half) * a.rows + r;
             if (row_ok) *reinterpret_cast<float2 *>(a.part_ml + rec * 2) = make_float2(m_ref, l_run);
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
@@ -680,27 +728,32 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
         // ---- this row's 64 scores (one TMEM load), log2 units, masked
         if (!FP8 && !mbar_wait(&s_full[j], (k >> 1) & 1)) break;
         tc_fence_after();
-        float x[64];
-        if (valid) tmem_ld64(tbase + lanes + j * 64, x);
+        float x[NT];
+        if (valid) {
+            if constexpr (FP8)
+                tmem_ld32(tbase + lanes + j * 64 + half * 32, x);
+            else
+                tmem_ld64(tbase + lanes + j * 64, x);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[j]);
         float alpha = 1.f;
-        uint32_t hw[32], lw[32];
+        uint32_t hw[NT / 2], lw[NT / 2];
         if (valid) {
             const int lim = min(L - 1, L - a.tq + t_r);   // last position the row sees
             const float sc = FP8 ? a.qscale * md.ks * q_inv : a.qscale * md.ks;
-            const int pos0 = md.j * kBlock;
+            const int pos0 = md.j * kBlock + half * 32;
             float mx = -INFINITY;
-            if (row_ok && pos0 + 63 <= lim) {   // the whole block is visible to the row
+            if (row_ok && pos0 + NT - 1 <= lim) {   // all of this thread's tokens are visible to the row
 #pragma unroll
-                for (int t = 0; t < 64; ++t) {
+                for (int t = 0; t < NT; ++t) {
                     x[t] *= sc;
                     mx = fmaxf(mx, x[t]);
                 }
             } else {
 #pragma unroll
-                for (int t = 0; t < 64; ++t) {
+                for (int t = 0; t < NT; ++t) {
                     x[t] = (row_ok && pos0 + t <= lim) ? x[t] * sc : -INFINITY;
                     mx = fmaxf(mx, x[t]);
                 }
@@ -719,7 +772,7 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
             const float mu = (m_ref == -INFINITY ? 0.f : m_ref) - lvs;
             float ps = 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < NT / 2; ++e) {
                 const float p0 = ex2_ftz(x[2 * e] - mu), p1 = ex2_ftz(x[2 * e + 1] - mu);
                 ps += p0 + p1;
                 if (FP8) {
@@ -751,13 +804,22 @@ __global__ void __launch_bounds__(kTcwThreads, 1)
                 rescale_o(a_o);
             }
             uint8_t *pb = pbuf + j * 16384;
+            if constexpr (FP8) {
+                // P row 64h + r, tokens 32h .. 32h + 31; the other half of the
+                // row stays zero (cleared at the start, never written)
+                const int prow = warp * 32 + lane;
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                *reinterpret_cast<uint4 *>(pb + sw128_offset(r, c8 * 8)) =
-                    make_uint4(hw[4 * c8], hw[4 * c8 + 1], hw[4 * c8 + 2], hw[4 * c8 + 3]);
-                if (!FP8)
+                for (int c8 = 0; c8 < 4; ++c8)
+                    *reinterpret_cast<uint4 *>(pb + sw128_offset(prow, half * 32 + c8 * 8)) =
+                        make_uint4(hw[4 * c8], hw[4 * c8 + 1], hw[4 * c8 + 2], hw[4 * c8 + 3]);
+            } else {
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    *reinterpret_cast<uint4 *>(pb + sw128_offset(r, c8 * 8)) =
+                        make_uint4(hw[4 * c8], hw[4 * c8 + 1], hw[4 * c8 + 2], hw[4 * c8 + 3]);
                     *reinterpret_cast<uint4 *>(pb + sw128_offset(64 + r, c8 * 8)) =
                         make_uint4(lw[4 * c8], lw[4 * c8 + 1], lw[4 * c8 + 2], lw[4 * c8 + 3]);
+                }
             }
             fence_proxy_async_smem();
             had_pv = true;

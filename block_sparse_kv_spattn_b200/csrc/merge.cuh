@@ -27,7 +27,7 @@ struct MergeArgs {
     float *lse;                 // nullable: [B][Tq][Hq], ln of the row's sum of exp(logit)
     int batch, tq, hq, hkv, group, rows, units, max_sel, ctas;
     int ntiles;                 // row tiles (units) per (request, KV head); rows = rows of one tile
-    int wslots;                 // partial records per (CTA, unit): 1 (attn_tcw) or 4 (one per attn_tc softmax warp)
+    int wslots;                 // partial records per (CTA, unit): 1 (attn_tcw, bf16), 2 (attn_tcw, fp8: two softmax halves) or 4 (one per attn_tc softmax warp)
     int pairs;                  // 4 records: warp w's pair w / 2 took only tiles of its parity
 };
 

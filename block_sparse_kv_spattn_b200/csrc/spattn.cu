@@ -155,7 +155,9 @@ bool uses_tc(const spattn_dims *d) { return d->kv_dtype == SPATTN_KV_BF16 && row
 
 // Partial records per (CTA, unit) slot: one per softmax warp (attn_tc), one
 // (attn_tcw).
-int records_per_slot(const spattn_dims *d) { return uses_tc(d) ? kTcWarpSlots : 1; }
+int records_per_slot(const spattn_dims *d) {
+    return uses_tc(d) ? kTcWarpSlots : tcw_records(d->kv_dtype == SPATTN_KV_FP8_E4M3);
+}
 
 // Per-device caches (SM count; which kernels have their shared-memory limit
 // raised).  Guarded by one mutex: these are host-side set-up calls only.
@@ -434,7 +436,7 @@ spattn_status launch_attn_tcw(AttnArgs &a, const void *k_cache, const void *v_ca
     SP_TRY(ensure_smem((const void *)attn_tcw_kernel<FP8>, smem));
     const int ctas = std::min(kMaxAttnCtas, sms);
     *ctas_out = ctas;
-    return cuda_ok(launch(attn_tcw_kernel<FP8>, dim3(ctas), dim3(kTcwThreads), smem, st, kmap, vmap, a),
+    return cuda_ok(launch(attn_tcw_kernel<FP8>, dim3(ctas), dim3(tcw_threads(FP8)), smem, st, kmap, vmap, a),
                    "attention (tensor core, many rows) launch");
 }
 

@@ -268,9 +268,9 @@ spattn_status spattn_decode_selected_lse(const spattn_dims *dims, const spattn_p
  * spattn_decode_selected; dims whose partial results need more than 16 MiB
  * ((320 + B * Hkv * T) x R x min(Tq * Hq / Hkv, 64) x (d + 2) x 4 bytes, T
  * = the 64-row tiles of a (request, KV head), R = 4 records per slot for
- * bf16 caches with Tq * Hq / Hkv <= 16, 1 otherwise) are rejected with
- * SPATTN_ERR_UNSUPPORTED before anything is enqueued.  No allocation call is
- * made.  The first call on each device looks up the array's device address
+ * bf16 caches with Tq * Hq / Hkv <= 16, 2 for fp8 caches, 1 otherwise) are
+ * rejected with SPATTN_ERR_UNSUPPORTED before anything is enqueued.  No
+ * allocation call is made.  The first call on each device looks up the array's device address
  * (a host-side CUDA runtime call), so make that first call before any stream
  * capture.  Every call on a device shares the one array and leaves its
  * contents behind; calls whose executions overlap on the GPU (different

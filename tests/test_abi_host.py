@@ -143,7 +143,7 @@ def test_hca_entry_points_validate_on_the_host(lib):
 @pytest.mark.parametrize("kw,records", [
     (dict(), 4),                                                  # bf16, 4 rows: one record per softmax warp
     (dict(q_tokens=4, num_q_heads=16, num_kv_heads=2), 1),        # 32 rows: the many-row kernel, one record
-    (dict(kv_dtype=1), 1),                                        # fp8: the many-row kernel
+    (dict(kv_dtype=1), 2),                                        # fp8: the many-row kernel, two softmax halves
 ])
 def test_workspace_size_is_the_documented_layout(lib, kw, records):
     """The scores (B x Tq x Hkv x max_blocks fp32) when spattn_decode keeps
