@@ -103,18 +103,22 @@ struct TcwMeta {
 // product reads them last): kMeta = kSrc + 8, see the producer.
 template <bool FP8>
 struct TcwLayout {
-    static constexpr int kOp = FP8 ? 2 : 4;          // bf16: stages; fp8: converted V buffers
-    static constexpr int kSrc = FP8 ? 5 : kOp;       // the ring the copies land in
+    static constexpr int kOp = FP8 ? 3 : 4;          // bf16: stages; fp8: converted V buffers
+    static constexpr int kSrc = FP8 ? 4 : kOp;       // the ring the copies land in
+    // P buffers (and their PV products): fp8 three, so that neither the
+    // softmax (writing P) nor the converters (writing V) wait for the PV
+    // product of the tile before the previous one
+    static constexpr int kPB = FP8 ? 3 : 2;
     static constexpr int kMeta = FP8 ? kSrc + 8 : kOp;
     // bf16: 64 rows x 128 bf16; fp8: the two e4m3 terms, each 128 rows (the
     // 64 query rows twice, for the two softmax halves) x 128 bytes
     static constexpr int kQSlot = FP8 ? 2 * 128 * 128 : kTcwRows * 256;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffP = kOffQ + 2 * kQSlot;                   // [2] P buffers
-    static constexpr int kOffK = kOffP + 2 * 128 * 128;                // bf16: K operands; fp8: the copy ring
+    static constexpr int kOffP = kOffQ + 2 * kQSlot;                   // [kPB] P buffers
+    static constexpr int kOffK = kOffP + kPB * 128 * 128;              // bf16: K operands; fp8: the copy ring
     static constexpr int kOffV = kOffK + kSrc * 16384;                 // V operands
     static constexpr int kOffMeta = kOffV + kOp * 16384;
-    static constexpr int kNBars = 2 * kSrc + kOp + 6 * 2 + 2;
+    static constexpr int kNBars = 2 * kSrc + kOp + 2 * kPB + 4 * 2 + 2;
     static constexpr int kOffBars = align16(kOffMeta + kMeta * (int)sizeof(TcwMeta));
     static constexpr int kSmem = align16(kOffBars + kNBars * 8 + 16);
 };
@@ -225,8 +229,8 @@ template <bool FP8>
 __global__ void __launch_bounds__(tcw_threads(FP8), 1)
     attn_tcw_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, AttnArgs a) {
     using TL = TcwLayout<FP8>;
-    constexpr int kOp = TL::kOp, kSrc = TL::kSrc, kMeta = TL::kMeta;
-    static_assert(!FP8 || kOp == 2, "fp8: V buffer of tile k is k & 1, the PV buffers' index");
+    constexpr int kOp = TL::kOp, kSrc = TL::kSrc, kMeta = TL::kMeta, kPB = TL::kPB;
+    static_assert(!FP8 || kOp == kPB, "fp8: V buffer of tile k is k % kPB, the PV buffers' index");
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *pbuf = smem + TL::kOffP;
     TcwMeta *meta = reinterpret_cast<TcwMeta *>(smem + TL::kOffMeta);
@@ -238,9 +242,9 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
     // be lapped by a phase two tiles ahead
     uint64_t *s_full = conv + kOp;              // [2] S buffer computed
     uint64_t *s_free = s_full + 2;              // [2] S buffer read (warps 0, 1)
-    uint64_t *p_full = s_free + 2;              // [2] P buffer written, rescales done (warps 0-3)
-    uint64_t *pv_done = p_full + 2;             // [2] the PV product of that buffer completed
-    uint64_t *q_free = pv_done + 2;             // [2] query slot's last product completed
+    uint64_t *p_full = s_free + 2;              // [kPB] P buffer written, rescales done (softmax warps)
+    uint64_t *pv_done = p_full + kPB;           // [kPB] the PV product of that buffer completed
+    uint64_t *q_free = pv_done + kPB;           // [2] query slot's last product completed
     uint64_t *q_read = q_free + 2;              // [2] fp8: the slot's row scales read (warps 0, 1)
     uint64_t *fin = q_read + 2;                 // MMA issuer: all products completed
     uint64_t *done = fin + 1;                   // warps 0-3 finished with TMEM
@@ -267,6 +271,8 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
             mbar_init(&s_free[p], tcw_softmax_warps(FP8));
             mbar_init(&q_free[p], 1);
             mbar_init(&q_read[p], tcw_softmax_warps(FP8));
+        }
+        for (int p = 0; p < kPB; ++p) {
             mbar_init(&p_full[p], tcw_softmax_warps(FP8));
             mbar_init(&pv_done[p], 1);
         }
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
     }
     if (FP8) {
         // the P halves a thread never writes stay zero
-        for (int i = threadIdx.x; i < 2 * 16384 / 16; i += blockDim.x)
+        for (int i = threadIdx.x; i < kPB * 16384 / 16; i += blockDim.x)
             reinterpret_cast<uint4 *>(pbuf)[i] = make_uint4(0u, 0u, 0u, 0u);
         fence_proxy_async_smem();
     }
@@ -478,8 +484,8 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
             if (!mbar_wait(&full[rs], (i / kSrc) & 1)) break;
             const TcwMeta m = meta[i % kMeta];
             if (FP8 && (m.flags & kEnd)) break;
-            // fp8: V buffer os is free once the PV product of tile i - 2 is done
-            if (FP8 && i >= 2 && !mbar_wait(&pv_done[os], ((i >> 1) - 1) & 1)) break;
+            // fp8: V buffer os is free once the PV product of tile i - kOp is done
+            if (FP8 && i >= kOp && !mbar_wait(&pv_done[os], ((i / kOp) - 1) & 1)) break;
             if (m.page >= 0) {
                 uint8_t *kop = smem + TL::kOffK + os * 16384, *vop = smem + TL::kOffV + os * 16384;
                 if (FP8) {
@@ -538,16 +544,16 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
             uint64_t t_idle = 0;
             while (pv < n) {
                 bool progressed = false;
-                if (pv < qk && mbar_test_wait(&p_full[pv & 1], (pv >> 1) & 1) &&
-                    (!FP8 || mbar_test_wait(&conv[pv & 1], (pv >> 1) & 1))) {   // first: a PV product frees a stage
+                if (pv < qk && mbar_test_wait(&p_full[pv % kPB], (pv / kPB) & 1) &&
+                    (!FP8 || mbar_test_wait(&conv[pv % kOp], (pv / kOp) & 1))) {   // first: a PV product frees a stage
                     tc_fence_after();
                     const int s = pv % kSrc;
                     const TcwMeta m = meta[pv % kMeta];
                     if (m.page >= 0) {
                         const uint32_t acc0 = last_seg == m.seg ? 1u : 0u;
                         last_seg = m.seg;
-                        const uint32_t vb = smem_u32(smem + TL::kOffV + (FP8 ? (pv & 1) : s) * 16384);
-                        const uint32_t pb = smem_u32(pbuf + (pv & 1) * 16384);
+                        const uint32_t vb = smem_u32(smem + TL::kOffV + (FP8 ? pv % kOp : s) * 16384);
+                        const uint32_t pb = smem_u32(pbuf + (pv % kPB) * 16384);
                         // O hi += P rows 0-63 . V ; O lo += P rows 64-127 . V (the
                         // other 64 lanes of each product are never read)
 #pragma unroll
@@ -559,10 +565,10 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
                                 umma_bf16(tbase + kTcwOLo, sw128_desc(pb + 8192 + ks * 32, 16, 1024), bd, kIdescPV,
                                           ks > 0 ? 1u : acc0);
                         }
-                        umma_commit(&pv_done[pv & 1]);
+                        umma_commit(&pv_done[pv % kPB]);
                         if (!FP8) umma_commit(&empty[s]);
                     } else {
-                        mbar_arrive(&pv_done[pv & 1]);
+                        mbar_arrive(&pv_done[pv % kPB]);
                         if (!FP8) mbar_arrive(&empty[s]);
                     }
                     ++pv;
@@ -653,7 +659,7 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
     int cur_seg = -1, unit = 0, L = 0, k_last = -1;
     bool had_pv = false;
     // wait for tile kk's PV products (its buffer's barrier)
-    auto wait_pv = [&](int kk) -> bool { return mbar_wait(&pv_done[kk & 1], (kk >> 1) & 1); };
+    auto wait_pv = [&](int kk) -> bool { return mbar_wait(&pv_done[kk % kPB], (kk / kPB) & 1); };
     auto rescale_o = [&](float f) {   // both parts of this row's accumulator
 #pragma unroll 1
         for (int cc = 0; cc < (FP8 ? 8 : 16); ++cc) {
@@ -794,8 +800,9 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
             l_run += md.vs == 1.f ? ps : ps / md.vs;
         }
         const float a_o = (valid && had_pv) ? alpha : 1.f;
-        // ---- P buffer j is free once tile k - 2's products are done
-        if (k >= 2 && !wait_pv(k - 2)) break;
+        // ---- P buffer k % kPB is free once tile k - kPB's products are done
+        const int jp = k % kPB;
+        if (k >= kPB && !wait_pv(k - kPB)) break;
         if (valid) {
             if (a_o != 1.f) {
                 // rescale this row's accumulator: after tile k - 1's products
@@ -803,7 +810,7 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
                 tc_fence_after();
                 rescale_o(a_o);
             }
-            uint8_t *pb = pbuf + j * 16384;
+            uint8_t *pb = pbuf + jp * 16384;
             if constexpr (FP8) {
                 // P row 64h + r, tokens 32h .. 32h + 31; the other half of the
                 // row stays zero (cleared at the start, never written)
@@ -826,7 +833,7 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[j]);
+        if (lane == 0) mbar_arrive(&p_full[jp]);
         k_last = k;
     }
     __syncwarp();
