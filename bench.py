@@ -313,10 +313,11 @@ def run_native(args, rank, world, local_rank):
                 spattn.hca_pool(kc, vc, ks, vs, bt, sl, khat, vhat, old_lens=old_lens, q_tokens=Tq)
         spattn.block_scores(q, kbar, bt, sl, scores, params, k_cache=kc)
         spattn.select(scores, sl, sel_idx, sel_count, params, q=q, k_cache=kc, block_table=bt)
+
+    def join_branches():   # the branches forked in front() (and the marks), before the step's end
         if not anchored:
             torch.cuda.current_stream().wait_stream(side)
-        if w.hca:
-            torch.cuda.current_stream().wait_stream(side2)
+        torch.cuda.current_stream().wait_stream(marks_stream)
 
     def attend():  # sparse attention + split merge
         if not w.hca:
@@ -326,20 +327,32 @@ def run_native(args, rank, world, local_rank):
 
     def hca():     # the HCA branch's attention and the merge of the two branches
         if w.hca:
+            torch.cuda.current_stream().wait_stream(side2)
             spattn.hca_attend(q, khat, vhat, sl, out, None, params, k_cache=kc, block_table=bt, workspace=hca_ws,
                               merge_with=(out_s, lse_s))
+
+    # the marks between the step's parts are recorded on a branch of their
+    # own, so that no kernel of the step waits behind an event node
+    marks_stream = torch.cuda.Stream()
+
+    def mark(ev):
+        marks_stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(marks_stream):
+            ev.record()
 
     # warm up eagerly once (sets kernel attributes), then capture graphs
     front()
     attend()
     hca()
+    join_branches()
     torch.cuda.synchronize()
     status = spattn.device_status()
     if status:
         raise RuntimeError(f"device status {status:#x}")
     # the whole step in one graph; events recorded as graph nodes time its
     # parts on the device (start, after the front, after the sparse
-    # attention, after the HCA branch)
+    # attention, after the HCA branch and the joins).  The middle two are
+    # leaves on a branch of their own (see mark()).
     marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -348,10 +361,11 @@ def run_native(args, rank, world, local_rank):
         with torch.cuda.graph(g_step, stream=s):
             marks[0].record()
             front()
-            marks[1].record()
+            mark(marks[1])
             attend()
-            marks[2].record()
+            mark(marks[2])
             hca()
+            join_branches()
             marks[3].record()
     torch.cuda.current_stream().wait_stream(s)
     kernels_error = None
@@ -364,7 +378,7 @@ def run_native(args, rank, world, local_rank):
     g_step.instantiate()
 
     K = args.steps
-    step_ms, attn_ms, hca_list = [], [], []
+    step_ms, attn_ms, hca_list, front_list = [], [], [], []
     props = torch.cuda.get_device_properties(dev)
     smi_id = (f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
               if hasattr(props, "pci_bus_id") else str(local_rank))
@@ -384,12 +398,13 @@ def run_native(args, rank, world, local_rank):
             step_ms.append(marks[0].elapsed_time(marks[3]))
             attn_ms.append(marks[1].elapsed_time(marks[2]))
             hca_list.append(marks[2].elapsed_time(marks[3]))
+            front_list.append(marks[0].elapsed_time(marks[1]))
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
         if world > 1:
             torch.distributed.barrier()
     hca_ms = sum(hca_list) / K
-    front_ms = sum(st - at - hc for st, at, hc in zip(step_ms, attn_ms, hca_list)) / K
+    front_ms = sum(front_list) / K
     total_ms = sum(step_ms)
     bts = step_bytes(inp, sel_count)
     status = spattn.device_status()

@@ -194,9 +194,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    // Launched early (programmatic dependent launch): nothing above reads
+    // global memory, as every input may come from the kernel before.  Once
+    // the wait returns, that kernel's writes (the selection) are final, so
+    // the merge behind this kernel may be scheduled: it reads only the
+    // selection counts before its own wait.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == 4) {
         // ============================================================ producer
+        const uint64_t kv_policy = l2_evict_first();
         int64_t W = 0;
         for (int u0 = 0; u0 < a.units; u0 += 32) {
             const int u = u0 + lane;
@@ -239,10 +247,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (page >= 0) {
                     const int y = (page * a.hkv + unit % a.hkv) * kBlock;
                     mbar_arrive_expect_tx(&full[s], kTcStageBytes);
-                    tma_load_2d(smem + TL::box(0, s), &kmap, 0, y, &full[s]);
-                    tma_load_2d(smem + TL::box(1, s), &kmap, 64, y, &full[s]);
-                    tma_load_2d(smem + TL::box(2, s), &vmap, 0, y, &full[s]);
-                    tma_load_2d(smem + TL::box(3, s), &vmap, 64, y, &full[s]);
+                    tma_load_2d(smem + TL::box(0, s), &kmap, 0, y, &full[s], kv_policy);
+                    tma_load_2d(smem + TL::box(1, s), &kmap, 64, y, &full[s], kv_policy);
+                    tma_load_2d(smem + TL::box(2, s), &vmap, 0, y, &full[s], kv_policy);
+                    tma_load_2d(smem + TL::box(3, s), &vmap, 64, y, &full[s], kv_policy);
                 } else {
                     mbar_arrive(&full[s]);
                 }

@@ -294,9 +294,17 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    // Launched early (programmatic dependent launch): nothing above reads
+    // global memory, as every input may come from the kernel before.  Once
+    // the wait returns, that kernel's writes (the selection) are final, so
+    // the merge behind this kernel may be scheduled: it reads only the
+    // selection counts before its own wait.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == 4) {
         // ============================================================ producer
+        const uint64_t kv_policy = l2_evict_first();
         int64_t W = 0;
         for (int u0 = 0; u0 < a.units; u0 += 32) {
             const int u = u0 + lane;
@@ -400,14 +408,14 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
                     const int y = (page * a.hkv + h) * kBlock;
                     if (FP8) {
                         mbar_arrive_expect_tx(&full[s], 2 * 8192);
-                        tma_load_2d(smem + TL::kOffK + s * 16384, &kmap, 0, y, &full[s]);   // codes: the operand
-                        tma_load_2d(smem + TL::kOffK + s * 16384 + 8192, &vmap, 0, y, &full[s]);
+                        tma_load_2d(smem + TL::kOffK + s * 16384, &kmap, 0, y, &full[s], kv_policy);   // codes: the operand
+                        tma_load_2d(smem + TL::kOffK + s * 16384 + 8192, &vmap, 0, y, &full[s], kv_policy);
                     } else {
                         mbar_arrive_expect_tx(&full[s], 4 * 8192);
-                        tma_load_2d(smem + TL::kOffK + s * 16384, &kmap, 0, y, &full[s]);
-                        tma_load_2d(smem + TL::kOffK + s * 16384 + 8192, &kmap, 64, y, &full[s]);
-                        tma_load_2d(smem + TL::kOffV + s * 16384, &vmap, 0, y, &full[s]);
-                        tma_load_2d(smem + TL::kOffV + s * 16384 + 8192, &vmap, 64, y, &full[s]);
+                        tma_load_2d(smem + TL::kOffK + s * 16384, &kmap, 0, y, &full[s], kv_policy);
+                        tma_load_2d(smem + TL::kOffK + s * 16384 + 8192, &kmap, 64, y, &full[s], kv_policy);
+                        tma_load_2d(smem + TL::kOffV + s * 16384, &vmap, 0, y, &full[s], kv_policy);
+                        tma_load_2d(smem + TL::kOffV + s * 16384 + 8192, &vmap, 64, y, &full[s], kv_policy);
                     }
                 } else {
                     mbar_arrive(&full[s]);

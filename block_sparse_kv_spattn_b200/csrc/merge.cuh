@@ -31,7 +31,8 @@ struct MergeArgs {
     int pairs;                  // 4 records: warp w's pair w / 2 took only tiles of its parity
 };
 
-constexpr int kMergeMaxWarps = 8;   // warps per output row, for units split over many CTAs
+constexpr int kMergeMaxWarps = 16;  // warps per output row, for units split over many CTAs
+constexpr int kMergeGroup = 16;     // records whose rows a warp loads together
 
 // Record x of a unit's candidate list (CTA c_lo + x / wslots, warp x %
 // wslots), or -1 if it was not written: the CTA's range misses the unit's
@@ -49,18 +50,24 @@ __host__ __device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int
     return ((int64_t)cc + unit) * a.wslots + w;
 }
 
-// One CTA per output row (b, t, query head): out = sum_s 2^(m_s - M) o_s /
-// sum_s 2^(m_s - M) l_s over the partial records of the row's unit: slot
-// c + unit for each CTA c whose range meets the unit's part of the sequence
-// (with wslots = 4, record w of that slot for each softmax warp w whose pair
-// took one of the CTA's tiles of the unit: pair w / 2 takes the tiles with
-// CTA-local index of its parity).  The CTA's warps take batches of 32
-// records in turn (a unit split over many CTAs has hundreds) and are
-// combined through shared memory.  A unit with nothing kept gets a zero row.
-__global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a) {
-    __shared__ float s_m[kMergeMaxWarps], s_l[kMergeMaxWarps];
-    __shared__ float4 s_acc[kMergeMaxWarps][32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+// One CTA of NW warps per output row (b, t, query head): out = sum_s
+// 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s over the partial records of the
+// row's unit: slot c + unit for each CTA c whose range meets the unit's part
+// of the sequence (with wslots = 4, record w of that slot for each softmax
+// warp w whose pair took one of the CTA's tiles of the unit: pair w / 2
+// takes the tiles with CTA-local index of its parity).  The warps take
+// groups of 16 records in turn (a unit split over many CTAs has hundreds),
+// each group's rows loaded together, and are combined through shared
+// memory.  A unit with nothing kept gets a zero row.
+//
+// Launched early behind the attention kernel (programmatic dependent
+// launch), which lets it be scheduled only once the selection is final: the
+// unit's place in the concatenated sequence and the warp's first records
+// are worked out from the selection counts before the wait, the records
+// themselves are read after it.
+template <int NW>
+__global__ void __launch_bounds__(NW * 32) merge_kernel(MergeArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t grow = blockIdx.x;
     const int i = (int)(grow % a.hq);
     const int t = (int)((grow / a.hq) % a.tq);
@@ -69,90 +76,93 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
     const int rg = t * a.group + g;                 // the row in the chunk's Tq * group
     const int unit = (b * a.hkv + h) * a.ntiles + rg / a.rows;
     const int row = rg % a.rows;
-    // prefix of the unit in the concatenated sequence, and the total W
+    // prefix of the unit in the concatenated sequence, and the total W (four
+    // count loads per lane in flight at a time)
     int64_t pre = 0, W = 0;
-    for (int u = lane; u < a.units; u += 32) {
-        const int cnt = min(max(a.sel_count[a.ntiles == 1 ? u : u / a.ntiles], 0), a.max_sel);
-        W += cnt;
-        if (u < unit) pre += cnt;
+    for (int u0 = 0; u0 < a.units; u0 += 128) {
+        int c4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int u = u0 + 32 * e + lane;
+            c4[e] = u < a.units ? a.sel_count[a.ntiles == 1 ? u : u / a.ntiles] : 0;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int cnt = min(max(c4[e], 0), a.max_sel);
+            W += cnt;
+            if (u0 + 32 * e + lane < unit) pre += cnt;
+        }
     }
     for (int o = 16; o > 0; o >>= 1) {
         pre += __shfl_xor_sync(0xffffffffu, pre, o);
         W += __shfl_xor_sync(0xffffffffu, W, o);
     }
     const int cnt = min(max(a.sel_count[unit / a.ntiles], 0), a.max_sel);
+    // records r = (slot * wslots + w) that were written: CTAs with an empty
+    // range (only when W < C) wrote none; with wslots = 4 a pair wrote only
+    // if it took a tile
+    int c_lo = 0, nrec = 0;
+    if (cnt > 0) {
+        c_lo = cta_of(pre, W, a.ctas);
+        nrec = (cta_of(pre + cnt - 1, W, a.ctas) - c_lo + 1) * a.wslots;
+    }
+    int x0 = warp * kMergeGroup;
+    int64_t r = lane < kMergeGroup && x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f, M = -INFINITY;
-    if (cnt > 0) {
-        // records r = (slot * wslots + w) that were written: CTAs with an
-        // empty range (only when W < C) wrote none; with wslots = 4 a pair
-        // wrote only if it took a tile
-        const int c_lo = cta_of(pre, W, a.ctas), c_hi = cta_of(pre + cnt - 1, W, a.ctas);
-        const int nrec = (c_hi - c_lo + 1) * a.wslots;
-        // batches of 32 records, one per lane, merged online.  A written
-        // record's row is finite even when its maximum is -inf (zero weights
-        // over zeroed unfilled slots), so the rows of the batch's first 16
-        // records are loaded together with the maxima, before the weights
-        // are known; a record that was not written reads a written one
-        // (weight 0).
-        for (int x0 = 32 * warp; x0 < nrec; x0 += 32 * nw) {
-            const int64_t r = x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
-            const unsigned written = __ballot_sync(0xffffffffu, r >= 0);
-            if (!written) continue;   // uniform
-            // (every lane takes part in the shuffle, then picks)
-            const int64_t rfirst = __shfl_sync(0xffffffffu, r, __ffs(written) - 1);
-            const int64_t rr = r >= 0 ? r : rfirst;
-            const int n_here = nrec - x0 < 32 ? nrec - x0 : 32;
-            float4 o16[16];
+    for (; x0 < nrec; x0 += NW * kMergeGroup) {
+        if (x0 != warp * kMergeGroup)
+            r = lane < kMergeGroup && x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
+        const unsigned written = __ballot_sync(0xffffffffu, r >= 0);
+        if (!written) continue;   // uniform
+        // A written record's row is finite even when its maximum is -inf
+        // (zero weights over zeroed unfilled slots), so the group's rows are
+        // loaded together with the maxima, before the weights are known; a
+        // record that was not written reads a written one (weight 0).
+        const int64_t rfirst = __shfl_sync(0xffffffffu, r, __ffs(written) - 1);
+        const int64_t rr = r >= 0 ? r : rfirst;
+        const int n_here = nrec - x0 < kMergeGroup ? nrec - x0 : kMergeGroup;
+        float4 o16[kMergeGroup];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int64_t re = __shfl_sync(0xffffffffu, rr, e);
-                o16[e] = e < n_here ? ld_f4_now(a.part_o + (re * a.rows + row) * kHeadDim + lane * 4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            float2 ml = make_float2(-INFINITY, 0.f);
-            if (r >= 0) ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
-            const float Mb = fmaxf(M, warp_max(ml.x));
-            const unsigned valid = __ballot_sync(0xffffffffu, r >= 0 && ml.x != -INFINITY);
-            // (no early exit here: the rows above stay in flight; a batch
-            // with nothing valid adds zero weights)
-            if (valid && Mb != M) {   // uniform: rescale what is summed so far
-                const float f = M == -INFINITY ? 0.f : exp2f(M - Mb);
-                acc.x *= f;
-                acc.y *= f;
-                acc.z *= f;
-                acc.w *= f;
-                lsum *= f;
-                M = Mb;
-            }
-            float w = 0.f;
-            if ((valid >> lane) & 1u) {
-                w = exp2f(ml.x - M);
-                lsum = fmaf(w, ml.y, lsum);
-            }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const float we = __shfl_sync(0xffffffffu, w, e);
-                acc.x = fmaf(we, o16[e].x, acc.x);
-                acc.y = fmaf(we, o16[e].y, acc.y);
-                acc.z = fmaf(we, o16[e].z, acc.z);
-                acc.w = fmaf(we, o16[e].w, acc.w);
-            }
-#pragma unroll 16
-            for (int e = 16; e < n_here; ++e) {
-                const float we = __shfl_sync(0xffffffffu, w, e);
-                const int64_t re = __shfl_sync(0xffffffffu, rr, e);
-                const float4 o = reinterpret_cast<const float4 *>(a.part_o + (re * a.rows + row) * kHeadDim)[lane];
-                acc.x = fmaf(we, o.x, acc.x);
-                acc.y = fmaf(we, o.y, acc.y);
-                acc.z = fmaf(we, o.z, acc.z);
-                acc.w = fmaf(we, o.w, acc.w);
-            }
+        for (int e = 0; e < kMergeGroup; ++e) {
+            const int64_t re = __shfl_sync(0xffffffffu, rr, e);
+            o16[e] = e < n_here ? ld_f4_now(a.part_o + (re * a.rows + row) * kHeadDim + lane * 4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        lsum = warp_sum(lsum);
+        float2 ml = make_float2(-INFINITY, 0.f);
+        if (r >= 0) ml = *reinterpret_cast<const float2 *>(a.part_ml + (r * a.rows + row) * 2);
+        const float Mb = fmaxf(M, warp_max(ml.x));
+        const unsigned valid = __ballot_sync(0xffffffffu, r >= 0 && ml.x != -INFINITY);
+        if (valid && Mb != M) {   // uniform: rescale what is summed so far
+            const float f = M == -INFINITY ? 0.f : exp2f(M - Mb);
+            acc.x *= f;
+            acc.y *= f;
+            acc.z *= f;
+            acc.w *= f;
+            lsum *= f;
+            M = Mb;
+        }
+        float w = 0.f;
+        if ((valid >> lane) & 1u) {
+            w = exp2f(ml.x - M);
+            lsum = fmaf(w, ml.y, lsum);
+        }
+#pragma unroll
+        for (int e = 0; e < kMergeGroup; ++e) {
+            const float we = __shfl_sync(0xffffffffu, w, e);
+            acc.x = fmaf(we, o16[e].x, acc.x);
+            acc.y = fmaf(we, o16[e].y, acc.y);
+            acc.z = fmaf(we, o16[e].z, acc.z);
+            acc.w = fmaf(we, o16[e].w, acc.w);
+        }
     }
-    if (nw > 1) {
+    lsum = warp_sum(lsum);
+    if constexpr (NW > 1) {
         // combine the warps: weights 2^(M_w - M)
+        __shared__ float s_m[NW], s_l[NW];
+        __shared__ float4 s_acc[NW][32];
         if (lane == 0) {
             s_m[warp] = M;
             s_l[warp] = lsum;
@@ -161,12 +171,13 @@ __global__ void __launch_bounds__(kMergeMaxWarps * 32) merge_kernel(MergeArgs a)
         __syncthreads();
         if (warp != 0) return;
         float Mt = -INFINITY;
-        for (int w = 0; w < nw; ++w) Mt = fmaxf(Mt, s_m[w]);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) Mt = fmaxf(Mt, s_m[w]);
         M = Mt;
         acc = make_float4(0.f, 0.f, 0.f, 0.f);
         lsum = 0.f;
         if (Mt != -INFINITY)
-            for (int w = 0; w < nw; ++w) {
+            for (int w = 0; w < NW; ++w) {
                 if (s_m[w] == -INFINITY) continue;
                 const float f = exp2f(s_m[w] - Mt);
                 const float4 o = s_acc[w][lane];

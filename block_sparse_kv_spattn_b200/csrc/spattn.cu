@@ -230,8 +230,7 @@ DecodeLayout decode_layout(const spattn_dims *d, bool with_scores) {
 
 // ------------------------------------------------------------- launches
 
-// Plain stream-ordered launch through cudaLaunchKernelEx.  (The split merge
-// after the attention kernel launched early was measured slower.)
+// Plain stream-ordered launch through cudaLaunchKernelEx.
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args &&...args) {
@@ -436,7 +435,7 @@ spattn_status launch_attn_tcw(AttnArgs &a, const void *k_cache, const void *v_ca
     SP_TRY(ensure_smem((const void *)attn_tcw_kernel<FP8>, smem));
     const int ctas = std::min(kMaxAttnCtas, sms);
     *ctas_out = ctas;
-    return cuda_ok(launch(attn_tcw_kernel<FP8>, dim3(ctas), dim3(tcw_threads(FP8)), smem, st, kmap, vmap, a),
+    return cuda_ok(launch_early(attn_tcw_kernel<FP8>, dim3(ctas), dim3(tcw_threads(FP8)), smem, st, kmap, vmap, a),
                    "attention (tensor core, many rows) launch");
 }
 
@@ -450,7 +449,7 @@ spattn_status launch_attn_tc_t(AttnArgs &a, const CUtensorMap &kmap, const CUten
     SP_TRY(ensure_smem(fn, smem));
     const int ctas = std::min(kMaxAttnCtas, sms);
     *ctas_out = ctas;
-    return cuda_ok(launch(attn_tc_kernel<RQ>, dim3(ctas), dim3(kTcThreads), smem, st, kmap, vmap, a),
+    return cuda_ok(launch_early(attn_tc_kernel<RQ>, dim3(ctas), dim3(kTcThreads), smem, st, kmap, vmap, a),
                    "attention (tensor core) launch");
 }
 
@@ -525,12 +524,21 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.wslots = records_per_slot(d);
     m.pairs = tc ? 1 : 0;
     // one CTA per output row; warps for the records a unit gets on average
-    // (CTAs per unit + 1, times the records per CTA), 32 per warp
+    // (CTAs per unit + 1, times the records per CTA), a group of 16 per warp
     const int64_t nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
     const int64_t recs = ((int64_t)ctas / std::max(1, a.units) + 2) * m.wslots;
     int wpr = 1;
-    while (wpr < kMergeMaxWarps && 32 * wpr < recs) wpr *= 2;
-    return cuda_ok(launch(merge_kernel, dim3((unsigned)nrows), dim3(32 * wpr), 0, st, m), "merge launch");
+    while (wpr < kMergeMaxWarps && kMergeGroup * wpr < recs) wpr *= 2;
+    const dim3 grid((unsigned)nrows), block(32 * wpr);
+    cudaError_t e;
+    switch (wpr) {
+        case 1: e = launch_early(merge_kernel<1>, grid, block, 0, st, m); break;
+        case 2: e = launch_early(merge_kernel<2>, grid, block, 0, st, m); break;
+        case 4: e = launch_early(merge_kernel<4>, grid, block, 0, st, m); break;
+        case 8: e = launch_early(merge_kernel<8>, grid, block, 0, st, m); break;
+        default: e = launch_early(merge_kernel<16>, grid, block, 0, st, m); break;
+    }
+    return cuda_ok(e, "merge launch");
 }
 
 spattn_status check_cache_args(const spattn_dims *d, const void *q, const void *k_cache,

@@ -106,12 +106,22 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
 
 // 2-D tiled tensor copy global -> shared, completion in bytes on `bar`.
 // x (innermost) must be a multiple of 16 bytes; here x is 0 or 64 bf16.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
+                                            uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-            "r"(smem_u32(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
+}
+
+// L2 policy for data a step reads once (the KV tiles): its lines are the
+// first to go, so that what the step reads again later (the partial
+// records, the selection) stays in L2 while the cache streams through.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
 // Bulk prefetch of [src, src + bytes) into L2 (no shared memory, no
