@@ -194,6 +194,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    // the lines (and translations) of the selection, the table and the
+    // lengths; prefetches use no data, so they may precede the wait
+    if (warp == 4) {
+        const int64_t nsel = (int64_t)(a.units / a.ntiles) * a.max_sel;
+        const int64_t nbt = (int64_t)(a.units / (a.ntiles * a.hkv)) * a.max_blocks;
+        const void *p[6] = {a.sel_count, a.sel_idx, a.sel_idx + (nsel > 0 ? nsel - 1 : 0), a.block_table,
+                            a.block_table + (nbt > 0 ? nbt - 1 : 0), a.seq_lens};
+        if (lane < 6) prefetch_l2(p[lane]);
+    }
     // Launched early (programmatic dependent launch): nothing above reads
     // global memory, as every input may come from the kernel before.  Once
     // the wait returns, that kernel's writes (the selection) are final, so
@@ -474,10 +483,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int r = 0; r < RQ; ++r) m_row = select_f((lane & 15) == r, m_ref[r], m_row);
             const int64_t rec = (((int64_t)c + unit) * kTcWarpSlots + warp) * a.rows;
-            if (lane < a.rows) {
-                a.part_ml[(rec + lane) * 2 + 0] = m_row;
-                a.part_ml[(rec + lane) * 2 + 1] = l_row;
-            }
+            const uint64_t keep = l2_evict_last();   // the merge reads the record next
+            if (lane < a.rows) st_global_f2(a.part_ml + (rec + lane) * 2, m_row, l_row, keep);
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 float v[16];
@@ -490,10 +497,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 16; ++e) v[e] += __shfl_xor_sync(0xffffffffu, v[e], 16);   // hi + lo
                 if (lane < a.rows) {
-                    float4 *dst = reinterpret_cast<float4 *>(a.part_o + (rec + lane) * kHeadDim + cc * 16);
+                    float *dst = a.part_o + (rec + lane) * kHeadDim + cc * 16;
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+                        st_global_f4(dst + 4 * e, v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3], keep);
                 }
             }
             tc_fence_before();

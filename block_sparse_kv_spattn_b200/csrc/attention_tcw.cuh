@@ -294,6 +294,15 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    // the lines (and translations) of the selection, the table and the
+    // lengths; prefetches use no data, so they may precede the wait
+    if (warp == 4) {
+        const int64_t nsel = (int64_t)(a.units / a.ntiles) * a.max_sel;
+        const int64_t nbt = (int64_t)(a.units / (a.ntiles * a.hkv)) * a.max_blocks;
+        const void *p[6] = {a.sel_count, a.sel_idx, a.sel_idx + (nsel > 0 ? nsel - 1 : 0), a.block_table,
+                            a.block_table + (nbt > 0 ? nbt - 1 : 0), a.seq_lens};
+        if (lane < 6) prefetch_l2(p[lane]);
+    }
     // Launched early (programmatic dependent launch): nothing above reads
     // global memory, as every input may come from the kernel before.  Once
     // the wait returns, that kernel's writes (the selection) are final, so
@@ -692,7 +701,8 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
             if (k_last >= 0 && !wait_pv(k_last)) break;
             tc_fence_after();
             const int64_t rec = (((int64_t)c + unit) * tcw_records(FP8) + half) * a.rows + r;
-            if (row_ok) *reinterpret_cast<float2 *>(a.part_ml + rec * 2) = make_float2(m_ref, l_run);
+            const uint64_t keep = l2_evict_last();   // the merge reads the record next
+            if (row_ok) st_global_f2(a.part_ml + rec * 2, m_ref, l_run, keep);
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 float v[16], w[16];
@@ -708,9 +718,10 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
                     for (int e = 0; e < 16; ++e) v[e] = 0.f;
                 }
                 if (row_ok) {
-                    float4 *dst = reinterpret_cast<float4 *>(a.part_o + rec * kHeadDim + cc * 16);
+                    float *dst = a.part_o + rec * kHeadDim + cc * 16;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+                    for (int e = 0; e < 4; ++e)
+                        st_global_f4(dst + 4 * e, v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3], keep);
                 }
             }
             tc_fence_before();

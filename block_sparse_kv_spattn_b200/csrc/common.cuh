@@ -157,6 +157,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Inclusive scan of an int over a warp.
+// L2 prefetch of the line holding p.  It uses no data, so a kernel launched
+// early may issue it before its wait on the kernel that writes p; its use is
+// that p's address translation and line are in place when p is accessed.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ int warp_incl_scan(int v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll

@@ -108,6 +108,12 @@ __global__ void __launch_bounds__(NW * 32) merge_kernel(MergeArgs a) {
     }
     int x0 = warp * kMergeGroup;
     int64_t r = lane < kMergeGroup && x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
+    // the records' lines (and translations) and the output row, before the wait
+    if (r >= 0) {
+        prefetch_l2(a.part_o + (r * a.rows + row) * kHeadDim);
+        prefetch_l2(a.part_ml + (r * a.rows + row) * 2);
+    }
+    if (warp == 0 && lane == 31) prefetch_l2(a.out + grow * kHeadDim);
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

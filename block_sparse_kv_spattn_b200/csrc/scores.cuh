@@ -84,7 +84,7 @@ __device__ __forceinline__ void load_kbar(const void *kbar, int page, int lane, 
 // Warp w takes blocks w, w + 4, ... of the CTA's range, BIF of them at a
 // time with all their compressed-key loads issued together.
 template <int HKV, bool KB16>
-__global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs a) {
+__global__ void __launch_bounds__(kScoreThreads, 5) block_scores_kernel(ScoresArgs a) {
     constexpr int BIF = HKV >= 16 ? 1 : (HKV >= 8 ? 2 : 4);
     constexpr int NW = kScoreThreads / 32;
     extern __shared__ float4 smem_f4[];
@@ -116,13 +116,13 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(ScoresArgs 
         const int hh = th % HKV, t = th / HKV;
         const uint16_t *qr = a.q + (((int64_t)b * a.tq + tb + t) * a.hq + hh * G) * kHeadDim + c8 * 8;
         float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int g0 = 0; g0 < G; g0 += 4) {  // the group's rows are loaded 4 at a time
-            uint4 u[4];
+        for (int g0 = 0; g0 < G; g0 += 8) {  // the group's rows are loaded 8 at a time
+            uint4 u[8];
 #pragma unroll
-            for (int gg = 0; gg < 4; ++gg)
+            for (int gg = 0; gg < 8; ++gg)
                 if (g0 + gg < G) u[gg] = *reinterpret_cast<const uint4 *>(qr + (g0 + gg) * kHeadDim);
 #pragma unroll
-            for (int gg = 0; gg < 4; ++gg) {
+            for (int gg = 0; gg < 8; ++gg) {
                 if (g0 + gg < G) {
                     float f[8];
                     bf16x8_to_f32(u[gg], f);

@@ -90,22 +90,22 @@ __device__ __forceinline__ float block_sum_f(float v, float *tmp) {
 }
 
 // Middle scores of a row -> order-preserving keys in shared memory.  The
-// row buffer has n_cap >= n readable columns, so the loads of a thread (8 at
-// a time) need not wait for n.  Returns the thread's max/min key over i < n.
+// row buffer has n_cap >= n readable columns, so the loads of a thread (16
+// at a time) need not wait for n.  Returns the thread's max/min key over i < n.
 __device__ __forceinline__ void load_keys(const SelectShared &sh, const float *row, int n_cap,
                                           const int *n_ptr, uint32_t &kmax, uint32_t &kmin) {
     kmax = 0;
     kmin = 0xffffffffu;
-    for (int i0 = threadIdx.x; i0 < n_cap; i0 += 8 * blockDim.x) {
-        float v[8];
+    for (int i0 = threadIdx.x; i0 < n_cap; i0 += 16 * blockDim.x) {
+        float v[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 16; ++u) {
             const int i = i0 + u * blockDim.x;
             v[u] = i < n_cap ? row[i] : 0.f;
         }
         const int n = *n_ptr;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 16; ++u) {
             const int i = i0 + u * blockDim.x;
             if (i < n) {
                 const uint32_t key = float_key(v[u]);
@@ -197,54 +197,6 @@ __device__ void radix_select(const SelectShared &sh, int n, int k, uint32_t &T, 
     need_eq = kk;
 }
 
-__device__ Cut find_cut(const SelectShared &sh, int n, int k, uint32_t kmax, uint32_t kmin) {
-    Cut cut{};
-    const float smax = key_float(kmax), smin = key_float(kmin);
-    if (isfinite(smax) && isfinite(smin) && smax > smin) {
-        cut.smin = smin;
-        cut.inv = (float)kBuckets / (smax - smin);
-        for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) sh.hist[i] = 0;
-        if (threadIdx.x == 0) sh.misc[3] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x)
-            atomicAdd(&sh.hist[bucket_of(key_float(sh.keys[i]), cut.smin, cut.inv)], 1u);
-        __syncthreads();
-        find_crossing(sh, kBuckets, k);
-        cut.bstar = sh.misc[0];
-        const int need = k - sh.misc[1], c = sh.misc[2];
-        if (c <= kCand) {
-            cut.bucket = true;
-            cut.ncand = c;
-            // gather the crossing bucket, then rank it exactly by (key desc, index asc)
-            for (int i = threadIdx.x; i < n; i += blockDim.x) {
-                const uint32_t key = sh.keys[i];
-                if (bucket_of(key_float(key), cut.smin, cut.inv) == cut.bstar) {
-                    const int slot = atomicAdd(&sh.misc[3], 1);
-                    sh.cand_key[slot] = key;
-                    sh.cand_idx[slot] = i;
-                }
-            }
-            __syncthreads();
-            for (int t = threadIdx.x; t < c; t += blockDim.x) {
-                const uint32_t kt = sh.cand_key[t];
-                const int it = sh.cand_idx[t];
-                int rank = 0;
-#pragma unroll 8
-                for (int u = 0; u < c; ++u) {
-                    const uint32_t ku = sh.cand_key[u];
-                    rank += ku > kt || (ku == kt && sh.cand_idx[u] < it);
-                }
-                sh.cand_ok[t] = rank < need;
-            }
-            __syncthreads();
-            return cut;
-        }
-    }
-    cut.bucket = false;
-    radix_select(sh, n, k, cut.T, cut.need_eq, cut.cnt_eq);
-    return cut;
-}
-
 // Visit the radix-form set {key > T} + {the first need_eq keys == T by
 // index} (contiguous index range per thread, one block scan).
 template <typename Fn>
@@ -275,6 +227,85 @@ __device__ void for_each_in_cut(const SelectShared &sh, int n, const Cut &cut, F
     } else {
         for_each_radix_chosen(sh, n, cut.T, cut.need_eq, fn);
     }
+}
+
+// The cut of the top k, and on_cut(i) called once for every element of it
+// (in no particular order).  on_each(i, key) is called once for every
+// element, in the order i = tid, tid + blockDim, ..., if and only if the
+// bucket form is tried; returns whether it was.  Bucket form: one histogram
+// pass (with on_each), then one pass that hands the elements of the buckets
+// above the crossing one to on_cut and gathers the crossing bucket, whose
+// candidates are ranked exactly by (key desc, index asc) and handed over by
+// thread t for candidate t.
+template <typename EachFn, typename CutFn>
+__device__ Cut find_cut(const SelectShared &sh, int n, int k, uint32_t kmax, uint32_t kmin, EachFn on_each,
+                        CutFn on_cut, bool *each_called) {
+    Cut cut{};
+    *each_called = false;
+    const float smax = key_float(kmax), smin = key_float(kmin);
+    if (isfinite(smax) && isfinite(smin) && smax > smin) {
+        *each_called = true;
+        cut.smin = smin;
+        cut.inv = (float)kBuckets / (smax - smin);
+        for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) sh.hist[i] = 0;
+        if (threadIdx.x == 0) sh.misc[3] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint32_t key = sh.keys[i];
+            on_each(i, key);
+            atomicAdd(&sh.hist[bucket_of(key_float(key), cut.smin, cut.inv)], 1u);
+        }
+        __syncthreads();
+        find_crossing(sh, kBuckets, k);
+        cut.bstar = sh.misc[0];
+        const int need = k - sh.misc[1], c = sh.misc[2];
+        if (c <= kCand) {
+            cut.bucket = true;
+            cut.ncand = c;
+            // the buckets above the crossing one go to on_cut; the crossing
+            // bucket is gathered
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                const uint32_t key = sh.keys[i];
+                const int bk = bucket_of(key_float(key), cut.smin, cut.inv);
+                if (bk > cut.bstar) {
+                    on_cut(i);
+                } else if (bk == cut.bstar) {
+                    const int slot = atomicAdd(&sh.misc[3], 1);
+                    sh.cand_key[slot] = key;
+                    sh.cand_idx[slot] = i;
+                }
+            }
+            __syncthreads();
+            // rank candidate t by four lanes of a warp, each over a quarter
+            // of the candidates (the warp's lanes stay together)
+            for (int base = threadIdx.x & ~31; base < 4 * c; base += blockDim.x) {
+                const int t4 = base + (threadIdx.x & 31);
+                const int t = t4 >> 2, part = t4 & 3;
+                int rank = 0;
+                if (t < c) {
+                    const uint32_t kt = sh.cand_key[t];
+                    const int it = sh.cand_idx[t];
+                    const int u_lo = part * c / 4, u_hi = (part + 1) * c / 4;
+#pragma unroll 4
+                    for (int u = u_lo; u < u_hi; ++u) {
+                        const uint32_t ku = sh.cand_key[u];
+                        rank += ku > kt || (ku == kt && sh.cand_idx[u] < it);
+                    }
+                }
+                rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+                rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+                if (t < c && part == 0) sh.cand_ok[t] = rank < need;
+            }
+            __syncthreads();
+            for (int t = threadIdx.x; t < c; t += blockDim.x)
+                if (sh.cand_ok[t]) on_cut(sh.cand_idx[t]);
+            return cut;
+        }
+    }
+    cut.bucket = false;
+    radix_select(sh, n, k, cut.T, cut.need_eq, cut.cnt_eq);
+    for_each_in_cut(sh, n, cut, on_cut);
+    return cut;
 }
 
 __device__ void bitonic_sort_desc(unsigned long long *buf, int N) {
@@ -375,24 +406,29 @@ __device__ void select_token(const SelectShared &sh, const SelectArgs &a, int b,
             return;
         }
     }
+    bool each_called;
     if (a.mode == SPATTN_SEL_TOPK) {
-        const Cut cut = find_cut(sh, n_mid, k, kmax, kmin);
-        for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });
+        find_cut(sh, n_mid, k, kmax, kmin, [](int, uint32_t) {}, [&](int i) { sh.flags[S + i] = 1; },
+                 &each_called);
         __syncthreads();
         return;
     }
-    // top-p: probabilities are the softmax of the middle scores
+    // top-p: probabilities are the softmax of the middle scores; the
+    // normaliser's terms are summed in the histogram pass when there is one
     const float smax = key_float(kmax);
-    float z = 0.f;
-    for (int i = threadIdx.x; i < n_mid; i += blockDim.x) z += expf(key_float(sh.keys[i]) - smax);
-    const float Z = block_sum_f(z, sh.ftmp);
+    float z = 0.f, mk = 0.f;
     Cut cut{};
+    each_called = false;
+    if (k < n_mid)   // mass of the k_max best blocks (mk) with the cut
+        cut = find_cut(
+            sh, n_mid, k, kmax, kmin, [&](int, uint32_t key) { z += expf(key_float(key) - smax); },
+            [&](int i) { mk += expf(key_float(sh.keys[i]) - smax); }, &each_called);
+    if (!each_called)
+        for (int i = threadIdx.x; i < n_mid; i += blockDim.x) z += expf(key_float(sh.keys[i]) - smax);
+    const float Z = block_sum_f(z, sh.ftmp);
     if (k < n_mid) {
-        cut = find_cut(sh, n_mid, k, kmax, kmin);
-        // mass of the k_max best blocks: below p, the cap decides alone
-        float m = 0.f;
-        for_each_in_cut(sh, n_mid, cut, [&](int i) { m += expf(key_float(sh.keys[i]) - smax); });
-        const float mass = block_sum_f(m, sh.ftmp) / Z;
+        // below p, the cap decides alone
+        const float mass = block_sum_f(mk, sh.ftmp) / Z;
         if (mass < a.top_p) {
             for_each_in_cut(sh, n_mid, cut, [&](int i) { sh.flags[S + i] = 1; });
             __syncthreads();
@@ -436,20 +472,42 @@ __device__ void select_token(const SelectShared &sh, const SelectArgs &a, int b,
     __syncthreads();
 }
 
-// Kept flags sh.flags[0, nb) -> ascending block ids of row bh.
+// Kept flags sh.flags[0, nb) -> ascending block ids of row bh.  Warp w
+// takes a run of consecutive 32-flag chunks (lane = flag, counted by
+// ballots); one scan over the warps' counts places the runs.
 __device__ void compact_flags(const SelectShared &sh, const SelectArgs &a, int bh, int nb) {
-    const int per = (nb + blockDim.x - 1) / blockDim.x;
-    const int lo = min(nb, (int)threadIdx.x * per), hi = min(nb, lo + per);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int nchunks = (nb + 31) >> 5;
+    const int per = (nchunks + nw - 1) / nw;
+    const int ch_lo = min(nchunks, warp * per), ch_hi = min(nchunks, ch_lo + per);
     int cnt = 0;
-    for (int j = lo; j < hi; ++j) cnt += sh.flags[j];
-    int total;
-    int pos = block_excl_scan(cnt, sh.itmp, &total);
+    for (int ch = ch_lo; ch < ch_hi; ++ch) {
+        const int j = ch * 32 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, j < nb && sh.flags[j]));
+    }
+    // (itmp is free: the caller's last barrier ended its previous use)
+    if (lane == 0) sh.itmp[warp] = cnt;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < nw ? sh.itmp[lane] : 0;
+        const int inc = warp_incl_scan(v);
+        __syncwarp();
+        if (lane < nw) sh.itmp[lane] = inc - v;
+        if (lane == 31) sh.itmp[32] = inc;
+    }
+    __syncthreads();
+    int pos = sh.itmp[warp];
+    const int total = sh.itmp[32];
     int32_t *dst = a.sel_idx + (int64_t)bh * a.max_sel;
-    for (int j = lo; j < hi; ++j)
-        if (sh.flags[j]) {
-            if (pos < a.max_sel) dst[pos] = j;
-            ++pos;
-        }
+    const unsigned below = (1u << lane) - 1u;
+    for (int ch = ch_lo; ch < ch_hi; ++ch) {
+        const int j = ch * 32 + lane;
+        const bool f = j < nb && sh.flags[j];
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        const int p = pos + __popc(bal & below);
+        if (f && p < a.max_sel) dst[p] = j;
+        pos += __popc(bal);
+    }
     if (threadIdx.x == 0) {
         if (total > a.max_sel) flag(SPATTN_DEV_SEL_OVERFLOW);
         a.sel_count[bh] = min(total, a.max_sel);
@@ -469,6 +527,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     // and itself started after every earlier kernel had finished, the
     // length is loaded before the wait.
     int L = a.len_early ? a.seq_lens[b] : 0;
+    // the lines (and translations) the kernel reads and writes, before the wait
+    if (threadIdx.x < 32) {
+        const int64_t last = (int64_t)a.tq * a.hkv * a.max_blocks - a.hkv * a.max_blocks;   // last token's row
+        const void *p[6] = {a.sel_idx + (int64_t)bh * a.max_sel, a.sel_idx + (int64_t)bh * a.max_sel + a.max_sel - 1,
+                            a.sel_count + bh, a.seq_lens + b,
+                            a.scores + ((int64_t)b * a.tq * a.hkv + h) * a.max_blocks,
+                            a.scores + ((int64_t)b * a.tq * a.hkv + h) * a.max_blocks + last + a.max_blocks - 1};
+        if (threadIdx.x < 6 && a.max_sel > 0) prefetch_l2(p[threadIdx.x]);
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (!a.len_early) L = a.seq_lens[b];
     // the first token's score row into L1

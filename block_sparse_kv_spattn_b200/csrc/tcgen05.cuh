@@ -124,6 +124,25 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
     return p;
 }
 
+// L2 policy for data the next kernel reads (the partial records): kept
+// longest, so that the cache streaming through L2 does not push it out.
+__device__ __forceinline__ uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Global stores with an L2 policy (p 16- / 8-byte aligned).
+__device__ __forceinline__ void st_global_f4(float *p, float a, float b, float c, float d, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d), "l"(policy)
+                 : "memory");
+}
+__device__ __forceinline__ void st_global_f2(float *p, float a, float b, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(a), "f"(b), "l"(policy)
+                 : "memory");
+}
+
 // Bulk prefetch of [src, src + bytes) into L2 (no shared memory, no
 // completion): src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void l2_prefetch(const void *src, uint32_t bytes) {
