@@ -61,6 +61,17 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+def _tensor_peak():
+    """Dense bf16 TFLOP/s sustained under the power cap (the attention is
+    timed inside a long run of steps)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops_sustained"]), "measured (MEASURED_PEAKS.json bf16_tflops_sustained)"
+    except Exception:
+        return 1400.0, "fallback"
+
+
 def attn_source_hash() -> str:
     h = hashlib.sha256()
     for f in ATTN_SOURCES:
@@ -194,6 +205,24 @@ def step_bytes(inp, sel_count: torch.Tensor) -> dict:
         hca = attend + pooled + len(lens) * H * D * 4 * 2
         d.update(hca=hca, hca_attend=attend, total=d["total"] + hca)
     return d
+
+
+def attention_flops(inp, sel_idx: torch.Tensor, sel_count: torch.Tensor) -> int:
+    """Algorithmic FLOPs of one sparse-attention launch: 4 d per (query row,
+    visible kept token) pair (q.k and p.v, 2 d each).  Query token t of a
+    chunk of Tq sits at position L - Tq + t and sees the kept positions up to
+    its own; every query head of the group sees the same ones."""
+    w = inp["workload"]
+    P, D, Tq = w.block_size, w.head_dim, w.q_tokens
+    G = w.num_q_heads // w.num_kv_heads
+    cnt, idx = sel_count.cpu(), sel_idx.cpu().to(torch.int64)
+    pairs = 0
+    for b, L in enumerate(inp["seq_lens"].tolist()):
+        lims = L - Tq + 1 + torch.arange(Tq, dtype=torch.int64)          # positions < lim are visible
+        for h in range(w.num_kv_heads):
+            start = idx[b, h, :int(cnt[b, h])] * P
+            pairs += int((lims[:, None] - start[None, :]).clamp(0, P).sum()) * G
+    return pairs * 4 * D
 
 
 def graph_kernels(g) -> list:
@@ -439,6 +468,12 @@ def run_native(args, rank, world, local_rank):
     attn_bytes = bts["kv"] + bts["q"] + bts["out"]     # one rank's launch
     achieved = attn_bytes / (attn_ms_mean * 1e-3) / 1e9
     traffic = measured_traffic(w, bts["kept_block_heads"])
+    # the attention's bound: its HBM bytes at the copy peak, or its FLOPs at
+    # the tensor peak, whichever takes longer
+    flops = attention_flops(inp, sel_idx, sel_count)
+    tpeak, tpeak_kind = _tensor_peak()
+    tensor_bound = flops / (tpeak * 1e12) > attn_bytes / (peak * 1e9)
+    tflops = flops / (attn_ms_mean * 1e-3) / 1e12
     queries = B * Tq * world / (ms_per_step * 1e-3)
     e2e_value = all_bytes / (e2e_total_ms / K * 1e-3) / 1e9
     line = {
@@ -450,12 +485,22 @@ def run_native(args, rank, world, local_rank):
         "hbm_fraction": round(value / peak, 4),
         "queries_per_s": round(queries, 1),
         "bytes_per_step": bts,
-        "roofline": {"kernel": attn_label(w),
-                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
-                     "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": None if traffic is None else int(traffic),
-                     "ms_per_launch": round(attn_ms_mean, 5)},
+        "roofline": ({"kernel": attn_label(w),
+                      "bound": "tensor", "achieved": round(tflops, 1), "peak": tpeak, "peak_kind": tpeak_kind,
+                      "unit": "TFLOP/s", "frac": round(tflops / tpeak, 4),
+                      "traffic": None if traffic is None else int(traffic),
+                      "ms_per_launch": round(attn_ms_mean, 5), "flops": flops,
+                      "hbm": {"achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                              "frac": round(achieved / peak, 4)}}
+                     if tensor_bound else
+                     {"kernel": attn_label(w),
+                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+                      "unit": "GB/s", "frac": round(achieved / peak, 4),
+                      "traffic": None if traffic is None else int(traffic),
+                      "ms_per_launch": round(attn_ms_mean, 5), "flops": flops,
+                      "tensor": {"achieved": round(tflops, 1), "peak": tpeak, "unit": "TFLOP/s",
+                                 "frac": round(tflops / tpeak, 4)}}),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": q.numel() * 2 + sl.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 4},
@@ -506,14 +551,19 @@ def kbar_recall(inp, params, sel_idx, sel_count, dev) -> float:
     return round(hit / max(1, total), 5)
 
 
-def oracle_request(inp, b, heads=None):
+def oracle_request(inp, b, heads=None, last_tokens=None):
     """The float64 oracle's work for request b of the batch: scores,
     selection and attention for all its KV heads, or only for the KV heads
     listed in `heads` (scores and selection still cover every head: they are
     a small part of the work); for the HCA workloads also the dense branch
-    and the merge.  Compressed keys and pooled entries are computed here,
-    outside the timed call, as the GPU step only re-compresses the appended
-    tail.  Returns run() -> kept block-heads of the attended heads."""
+    and the merge.  `last_tokens`: the attention of a chunk's last n query
+    tokens only (at their own positions, over the selection of the whole
+    chunk).  Compressed keys and pooled entries are computed here, outside
+    the timed call, as the GPU step only re-compresses the appended tail.
+    Returns run() -> kept block-heads of the attended heads."""
+    import dataclasses
+
+    import numpy as np
     import oracle
     from oracle.marshal import bits16, cache_bytes, dims_of, params_of, subproblem
 
@@ -527,11 +577,16 @@ def oracle_request(inp, b, heads=None):
     kbar = oracle.compress_keys(dims, kh, ksc, bt, sl)
     hat = oracle.hca_pool(dims, kh, vh, ksc, vsc, bt, sl) if w.hca else None
     units = None if heads is None else [(0, h) for h in heads]
+    dims_a, q_a = dims, qh
+    if last_tokens is not None and last_tokens < w.q_tokens:
+        # token t' of the last n sits at L - n + t' = L - Tq + (Tq - n + t')
+        dims_a = dataclasses.replace(dims, q_tokens=last_tokens)
+        q_a = np.ascontiguousarray(qh[:, w.q_tokens - last_tokens:])
 
     def run():
         sc = oracle.block_scores(dims, par, qh, kbar, bt, sl)
         sel, cnt, _ = oracle.select(dims, par, sc, sl)
-        o_s = oracle.attend(dims, par, qh, kh, vh, ksc, vsc, bt, sl, sel, cnt, with_lse=w.hca, units=units)
+        o_s = oracle.attend(dims_a, par, q_a, kh, vh, ksc, vsc, bt, sl, sel, cnt, with_lse=w.hca, units=units)
         if w.hca:
             oracle.lse_merge(*o_s, *oracle.hca_attend(dims, par, qh, hat[0], hat[1], sl))
         return int(cnt.sum()) if heads is None else int(sum(cnt[0, h] for h in heads))
@@ -553,20 +608,26 @@ def cpu_baseline(inp, bts, gpu_ms):
     """The float64 oracle on this host's cores, on a bounded sample: request
     0 (scores, selection, attention), about 10 s of runs on every core,
     scaled to the whole step.  When one request would take more than ~10 s,
-    the sample is its KV head 0 alone (scaled by the KV heads too).  Then a
-    few runs on one core, when they fit in ~30 s."""
+    the sample is its KV head 0 alone (scaled by the KV heads too), and when
+    that would too (long prefill chunks), the attention of the chunk's last
+    few query tokens of KV head 0 (scaled by the tokens too).  Then a few
+    runs on one core, when they fit in ~30 s."""
     import oracle
 
     w = inp["workload"]
-    H = w.num_kv_heads
+    H, Tq = w.num_kv_heads, w.q_tokens
     cores = oracle.num_threads()
-    probe = oracle_request(inp, 0, heads=[0])
-    t_unit = min(_time_runs(probe, 0.0, min_runs=1, max_runs=1))
+    # one query token of KV head 0: the whole unit is at most Tq times that
+    t_tok = min(_time_runs(oracle_request(inp, 0, heads=[0], last_tokens=1), 0.0, min_runs=1, max_runs=1))
+    t_unit = t_tok * Tq
     whole = w.hca or H == 1 or t_unit * H <= 10.0   # (the HCA branch covers every head at once)
-    run = oracle_request(inp, 0) if whole else probe
-    scale = w.batch if whole else w.batch * H
+    n_tok = Tq if t_unit <= 10.0 else max(1, min(Tq, int(10.0 / t_tok)))
+    run = oracle_request(inp, 0) if whole else oracle_request(inp, 0, heads=[0], last_tokens=n_tok)
+    scale = w.batch if whole else w.batch * H * Tq / n_tok
     what = (f"request 0 of {w.batch} (all {H} KV heads{', both branches' if w.hca else ''})" if whole
-            else f"KV head 0 of request 0 (one of {w.batch * H} (request, KV head) units)")
+            else f"KV head 0 of request 0 (one of {w.batch * H} (request, KV head) units)" if n_tok == Tq
+            else (f"the last {n_tok} of {Tq} query tokens of KV head 0 of request 0 (one of {w.batch * H} "
+                  f"(request, KV head) units; selection over the whole chunk)"))
     times = _time_runs(run, 10.0)
     per = statistics.median(times)
     step_s = per * scale
@@ -575,7 +636,7 @@ def cpu_baseline(inp, bts, gpu_ms):
     used = min(cores, H if whole else 1)
     line = {"value": round(bts["total"] / step_s / 1e9, 4), "unit": "GB/s", "cores": used,
             "host_threads": cores, "kind": "oracle",
-            "sample": f"{what}, {len(times)} runs, median {per:.3f} s, scaled x{scale} to the step",
+            "sample": f"{what}, {len(times)} runs, median {per:.3f} s, scaled x{scale:g} to the step",
             "ms_per_step": round(step_s * 1e3, 3), "gpu_speedup": round(step_s * 1e3 / gpu_ms, 1)}
     # one core: the same sample, if about 5 runs fit in ~30 s
     if per * used * 5 <= 30.0 or used == 1:
@@ -587,7 +648,7 @@ def cpu_baseline(inp, bts, gpu_ms):
         step1_s = statistics.median(t1) * scale
         line["one_core"] = {"value": round(bts["total"] / step1_s / 1e9, 5), "unit": "GB/s", "cores": 1,
                             "ms_per_step": round(step1_s * 1e3, 3),
-                            "sample": f"the same sample, {len(t1)} runs on one thread, scaled x{scale}"}
+                            "sample": f"the same sample, {len(t1)} runs on one thread, scaled x{scale:g}"}
     return line
 
 

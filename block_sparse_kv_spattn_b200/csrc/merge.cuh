@@ -32,7 +32,10 @@ struct MergeArgs {
 };
 
 constexpr int kMergeMaxWarps = 16;  // warps per output row, for units split over many CTAs
-constexpr int kMergeGroup = 16;     // records whose rows a warp loads together
+
+// Records whose rows a warp loads together: 16, or 20 with the most warps
+// (a unit spread over the whole grid, about 300 records, in one round).
+__host__ __device__ constexpr int merge_group(int nw) { return nw >= kMergeMaxWarps ? 20 : 16; }
 
 // Record x of a unit's candidate list (CTA c_lo + x / wslots, warp x %
 // wslots), or -1 if it was not written: the CTA's range misses the unit's
@@ -56,17 +59,18 @@ __host__ __device__ __forceinline__ int64_t merge_record(const MergeArgs &a, int
 // of the sequence (with wslots = 4, record w of that slot for each softmax
 // warp w whose pair took one of the CTA's tiles of the unit: pair w / 2
 // takes the tiles with CTA-local index of its parity).  The warps take
-// groups of 16 records in turn (a unit split over many CTAs has hundreds),
-// each group's rows loaded together, and are combined through shared
-// memory.  A unit with nothing kept gets a zero row.
+// groups of 16 records in turn (20 with 16 warps; a unit split over many
+// CTAs has hundreds), each group's rows loaded together, and are combined
+// through shared memory.  A unit with nothing kept gets a zero row.
 //
 // Launched early behind the attention kernel (programmatic dependent
 // launch), which lets it be scheduled only once the selection is final: the
 // unit's place in the concatenated sequence and the warp's first records
-// are worked out from the selection counts before the wait, the records
-// themselves are read after it.
+// are worked out from the selection counts before the wait (and their lines
+// prefetched), the records themselves are read after it.
 template <int NW>
 __global__ void __launch_bounds__(NW * 32) merge_kernel(MergeArgs a) {
+    constexpr int kMergeGroup = merge_group(NW);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t grow = blockIdx.x;
     const int i = (int)(grow % a.hq);
@@ -109,9 +113,13 @@ __global__ void __launch_bounds__(NW * 32) merge_kernel(MergeArgs a) {
     int x0 = warp * kMergeGroup;
     int64_t r = lane < kMergeGroup && x0 + lane < nrec ? merge_record(a, x0 + lane, c_lo, unit, pre, cnt, W) : -1;
     // the records' lines (and translations) and the output row, before the wait
-    if (r >= 0) {
-        prefetch_l2(a.part_o + (r * a.rows + row) * kHeadDim);
-        prefetch_l2(a.part_ml + (r * a.rows + row) * 2);
+    for (int xp = x0; xp < nrec; xp += NW * kMergeGroup) {
+        const int64_t rp = xp == x0 ? r : (lane < kMergeGroup && xp + lane < nrec
+                                               ? merge_record(a, xp + lane, c_lo, unit, pre, cnt, W) : -1);
+        if (rp >= 0) {
+            prefetch_l2(a.part_o + (rp * a.rows + row) * kHeadDim);
+            prefetch_l2(a.part_ml + (rp * a.rows + row) * 2);
+        }
     }
     if (warp == 0 && lane == 31) prefetch_l2(a.out + grow * kHeadDim);
     asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -524,11 +524,11 @@ spattn_status launch_attention(const spattn_dims *d, const spattn_params *p, con
     m.wslots = records_per_slot(d);
     m.pairs = tc ? 1 : 0;
     // one CTA per output row; warps for the records a unit gets on average
-    // (CTAs per unit + 1, times the records per CTA), a group of 16 per warp
+    // (CTAs per unit + 1, times the records per CTA), a group of 16 or 20 per warp
     const int64_t nrows = (int64_t)d->batch * d->q_tokens * d->num_q_heads;
     const int64_t recs = ((int64_t)ctas / std::max(1, a.units) + 2) * m.wslots;
     int wpr = 1;
-    while (wpr < kMergeMaxWarps && kMergeGroup * wpr < recs) wpr *= 2;
+    while (wpr < kMergeMaxWarps && merge_group(wpr) * wpr < recs) wpr *= 2;
     const dim3 grid((unsigned)nrows), block(32 * wpr);
     cudaError_t e;
     switch (wpr) {

@@ -120,6 +120,12 @@ WORKLOADS = {
     "chunk16_fp8_128k": Workload("chunk16_fp8_128k", batch=4, q_tokens=16, num_q_heads=32,
                                  num_kv_heads=8, seq_len=131072, kv_fp8=True, structure="zipf",
                                  mode="topk", max_ratio=0.12, seed=1242),
+    # a prefill chunk: 64 tokens x 8 query heads per KV head = 512 query rows
+    # per (request, KV head), eight 64-row tiles over the chunk's union
+    # selection (top-k 10 % per token), bf16 cache
+    "prefill_chunk64_128k": Workload("prefill_chunk64_128k", batch=2, q_tokens=64, num_q_heads=64,
+                                     num_kv_heads=8, seq_len=131072, structure="zipf", mode="topk",
+                                     max_ratio=0.10, seed=1243),
 }
 
 BENCH_WORKLOAD = "decode_128k_b8"
