@@ -218,11 +218,16 @@ size_t spattn_decode_workspace_size(const spattn_dims *dims, const spattn_params
  * fp32 accumulation; split-KV partials merged by their log-sum-exp).
  * A row with no visible token is all zeros.  sel_idx / sel_count as written
  * by spattn_select (any ascending or unordered list of distinct ids works).
- * Both kernels run on the tensor cores (tcgen05, probabilities entered as
- * bf16 hi + lo parts): bf16 caches with Tq * Hq / Hkv <= 16 with the tokens
- * of a block on M; fp8 caches (codes widened to bf16 in shared memory, the
- * scales applied to the scores and the weights) and larger row counts with
- * the query rows on M.
+ * Both kernels run on the tensor cores (tcgen05): bf16 caches with
+ * Tq * Hq / Hkv <= 16 with the tokens of a block on M (probabilities
+ * entered as bf16 hi + lo parts); fp8 caches and larger row counts with the
+ * query rows on M, in 64-row tiles (fp8: the scores from the key codes as
+ * stored and the query split into two exact e4m3 terms, the values widened
+ * e4m3 -> f16 exactly and weighted in f16; the scales applied to the scores
+ * and the weights).  The kernels are launched with programmatic dependent
+ * launch: each waits for the kernel before it in the stream to complete
+ * before it reads any argument's memory, so inputs written by that kernel
+ * are seen.
  */
 spattn_status spattn_decode_selected(const spattn_dims *dims, const spattn_params *params,
                                      const void *q, const void *k_cache, const void *v_cache,
