@@ -27,8 +27,10 @@ struct ScoresArgs {
 constexpr int kScoreThreads = 128;
 
 // Blocks per CTA: small CTAs (many resident per SM, many loads in flight)
-// unless the query rows make the per-CTA q-bar prologue heavy.
-__host__ __device__ constexpr int score_blocks_per_cta(int rows) { return rows <= 16 ? 16 : 64; }
+// unless the query rows make the per-CTA q-bar prologue heavy, or there are
+// so few rows (one or two KV heads of a decode step) that a CTA's compressed
+// keys are a short read beside its prologue.
+__host__ __device__ constexpr int score_blocks_per_cta(int rows) { return rows <= 2 ? 64 : (rows <= 16 ? 16 : 64); }
 static_assert(score_blocks_per_cta(1) <= kScoreThreads && score_blocks_per_cta(64) <= kScoreThreads,
               "one block-table entry per thread");
 
