@@ -1,6 +1,6 @@
 // attention_tcw.cuh -- exact softmax attention over the kept blocks on the
 // sm_100a tensor cores for many query rows per KV head (a chunk of tokens
-// times the group's heads, up to 64) and for fp8 caches.
+// times the group's heads, in tiles of 64 rows) and for fp8 caches.
 //
 // "CSA + HCA 混合注意力机制" §2.1 / §4.4 step 4: softmax(q K_sel^T / sqrt(d)) V_sel
 // over the selected entries only; §4.3: the window and the partly filled
@@ -8,10 +8,12 @@
 // stored as fp8 with a scale per (page, KV head).
 //
 // Work split, segments and records follow attention.cuh: the kept lists of
-// all (request, KV head) units are concatenated and cut into equal ranges,
-// one per CTA of a persistent grid.
+// all units are concatenated and cut into equal ranges, one per CTA of a
+// persistent grid; a unit is one 64-row tile of a (request, KV head), so a
+// longer chunk runs as several units over the same kept blocks, each masked
+// by its own rows' tokens.
 //
-// Products per kept block (64 tokens), query rows on M:
+// Products per kept block (64 tokens), query rows on M, bf16 caches:
 //   S [128 x 64]   = Q [128 x d] . K^T      K-major A (query slot) and B (the
 //                    block's keys).  Rows 0-63 are the unit's query rows
 //                    (zero padded); rows 64-127 read whatever follows the
@@ -31,16 +33,26 @@
 // row are rescaled).  One partial record (m, l, O = hi + lo) per row and
 // segment.
 //
-// fp8 caches: the bulk copies land in a staging buffer and converter warps
-// widen the codes to bf16 (exact: every e4m3 value is a bf16 value) into the
-// operand layout; the per-(page, KV head) scales multiply the scores (K) and
-// the weights (V).  bf16 caches are copied straight into the operand layout
-// by TMA.  Either way the converter warps zero the V rows of unfilled token
-// slots, so that zero weights never meet non-finite values.
+// fp8 caches: the copies land in a ring of [K codes | V codes] stages.  The
+// QK product runs in kind::f8f6f4 on the key codes as copied: each query row
+// is scaled by a power of two (its largest element in [2^7, 2^8)) and split
+// into two e4m3 terms q1 + q2, exact for every element within 2^9 of the
+// row's largest, so S = q1 . K + q2 . K (the slot holds each term's 64 rows
+// twice, rows r and 64 + r, so lanes 64-127 carry the same scores).
+// Converter warps widen the V codes to f16 (exact) into their own buffers,
+// and PV runs in f16 with one f16 weight per element (the reference maximum
+// follows x + log2 s_v, so every weight stays below 2^15).  The softmax runs
+// in two halves (tokens 0-31 and 32-63 of a block), each with its own
+// reference maximum, sums, output rows and partial record.  The per-(page,
+// KV head) scales multiply the scores (K) and the weights (V).  bf16 caches
+// are copied straight into the operand layout by TMA.  Either way the
+// converter warps zero the V rows of unfilled token slots, so that zero
+// weights never meet non-finite values.
 //
-// Warps: 0-1 softmax (query rows 0-63; TMEM lanes 0-63), 4 producer, 5 MMA
-// issue (one lane) and TMEM owner, 2, 3, 6, 7 converters.  Every wait is
-// bounded (SPATTN_DEV_WAIT_TIMEOUT).
+// Warps, bf16 caches: 0-1 softmax (query rows 0-63; TMEM lanes 0-63), 4
+// producer, 5 MMA issue (one lane) and TMEM owner, 2, 3, 6, 7 converters;
+// fp8 caches: 0-3 softmax, 4 producer, 5 MMA issue, 6-9 converters.  Every
+// wait is bounded (SPATTN_DEV_WAIT_TIMEOUT).
 #pragma once
 
 #include "attention.cuh"
@@ -87,7 +99,7 @@ struct TcwMeta {
 };
 
 // Shared memory: two query slots (64 rows x 128 bf16 as two 64-column halves,
-// or the two e4m3 terms of the rows), two P buffers (128 rows x 64 bf16 or
+// or the two e4m3 terms of the rows), kPB P buffers (128 rows x 64 bf16 or
 // f16), the copy stages and operands below, then meta and barriers.  Operand
 // tiles on 1024-byte boundaries.
 //
@@ -96,7 +108,7 @@ struct TcwMeta {
 // product is done.
 // fp8 caches: a ring of kSrc copy stages, each [K codes 8 KB | V codes 8
 // KB] of one block (the K codes are the QK operand as copied), released once
-// the block's QK product is done and its V codes are converted; and kOp = 2
+// the block's QK product is done and its V codes are converted; and kOp = 3
 // buffers of converted V (f16 operand), released by the PV product.  A copy
 // stage therefore lives for the copy, QK and the conversion only, so that
 // many blocks' copies are in flight.  Meta entries outlive the stage (the PV
@@ -122,19 +134,6 @@ struct TcwLayout {
     static constexpr int kOffBars = align16(kOffMeta + kMeta * (int)sizeof(TcwMeta));
     static constexpr int kSmem = align16(kOffBars + kNBars * 8 + 16);
 };
-
-// Two e4m3 codes (low byte first) -> two bf16 (low half first), exactly:
-// the hardware e4m3x2 -> f16x2 conversion, then f16 -> bf16 by moving the
-// fields (every e4m3 value is a normal f16 or zero, with at most 3 mantissa
-// bits): magnitude >> 3 puts exponent and mantissa in place, + 112 << 7
-// rebiases the exponent for the nonzero halves, and the sign stays.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes) {
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(codes & 0xffffu)));
-    const uint32_t mag = (h2 >> 3) & 0x0fff0fffu;               // 0, or >= 0x300 (2^-9) per half
-    const uint32_t nz = ((mag + 0x0d000d00u) & 0x10001000u) >> 12;   // 1 per nonzero half
-    return (nz * 0x3800u + mag) | (h2 & 0x80008000u);
-}
 
 // Two e4m3 codes (low byte first) -> two f16 (low half first): one hardware
 // conversion, exact (every e4m3 value is an f16 value).
@@ -504,32 +503,23 @@ __global__ void __launch_bounds__(tcw_threads(FP8), 1)
             // fp8: V buffer os is free once the PV product of tile i - kOp is done
             if (FP8 && i >= kOp && !mbar_wait(&pv_done[os], ((i / kOp) - 1) & 1)) break;
             if (m.page >= 0) {
-                uint8_t *kop = smem + TL::kOffK + os * 16384, *vop = smem + TL::kOffV + os * 16384;
+                uint8_t *vop = smem + TL::kOffV + os * 16384;
                 if (FP8) {
                     const uint8_t *stg = smem + TL::kOffK + rs * 16384;   // [K codes | V codes]
 #pragma unroll
                     for (int e = 0; e < 512 / (kTcwConvWarps * 32); ++e) {
-                        const int task = 512 + ct + e * kTcwConvWarps * 32;   // V only (K is used as copied)
-                        const bool isv = task >= 512;
+                        // V only (the K codes are the QK operand as copied)
+                        const int task = ct + e * kTcwConvWarps * 32;
                         const int tt = task & 63, c16 = (task >> 6) & 7;   // token, 16-column chunk
-                        const uint4 u = *reinterpret_cast<const uint4 *>(stg + (isv ? 8192 : 0) + tt * 128 +
+                        const uint4 u = *reinterpret_cast<const uint4 *>(stg + 8192 + tt * 128 +
                                                                          ((c16 ^ (tt & 7)) << 4));
-                        // K to bf16 (the QK product's type); V to f16 (the PV
-                        // product takes f16 weights and values: one conversion)
-                        uint4 w0, w1;
-                        if (isv) {
-                            w0 = make_uint4(e4m3x2_to_f16x2(u.x), e4m3x2_to_f16x2(u.x >> 16),
-                                            e4m3x2_to_f16x2(u.y), e4m3x2_to_f16x2(u.y >> 16));
-                            w1 = make_uint4(e4m3x2_to_f16x2(u.z), e4m3x2_to_f16x2(u.z >> 16),
-                                            e4m3x2_to_f16x2(u.w), e4m3x2_to_f16x2(u.w >> 16));
-                        } else {
-                            w0 = make_uint4(e4m3x2_to_bf16x2(u.x), e4m3x2_to_bf16x2(u.x >> 16),
-                                            e4m3x2_to_bf16x2(u.y), e4m3x2_to_bf16x2(u.y >> 16));
-                            w1 = make_uint4(e4m3x2_to_bf16x2(u.z), e4m3x2_to_bf16x2(u.z >> 16),
-                                            e4m3x2_to_bf16x2(u.w), e4m3x2_to_bf16x2(u.w >> 16));
-                        }
-                        if (isv && tt >= m.nvalid) w0 = w1 = make_uint4(0u, 0u, 0u, 0u);
-                        uint8_t *box = (isv ? vop : kop) + (c16 >> 2) * 8192;
+                        // to f16: the PV product takes f16 weights and values
+                        uint4 w0 = make_uint4(e4m3x2_to_f16x2(u.x), e4m3x2_to_f16x2(u.x >> 16),
+                                              e4m3x2_to_f16x2(u.y), e4m3x2_to_f16x2(u.y >> 16));
+                        uint4 w1 = make_uint4(e4m3x2_to_f16x2(u.z), e4m3x2_to_f16x2(u.z >> 16),
+                                              e4m3x2_to_f16x2(u.w), e4m3x2_to_f16x2(u.w >> 16));
+                        if (tt >= m.nvalid) w0 = w1 = make_uint4(0u, 0u, 0u, 0u);
+                        uint8_t *box = vop + (c16 >> 2) * 8192;
                         const int col = (c16 & 3) * 16;
                         *reinterpret_cast<uint4 *>(box + sw128_offset(tt, col)) = w0;
                         *reinterpret_cast<uint4 *>(box + sw128_offset(tt, col + 8)) = w1;
