@@ -197,7 +197,10 @@ spattn_status spattn_block_scores(const spattn_dims *dims, const spattn_params *
  * Reads scores as written by spattn_block_scores (only the middle columns
  * are read) and writes the ascending kept block ids of (b, h) to
  * sel_idx[b][h][0 .. sel_count[b][h]).  Top-p probabilities and their running
- * sum are fp32.
+ * sum are fp32.  Launched with programmatic dependent launch: the kernel
+ * waits for the kernel before it in the stream to complete before it reads
+ * any argument's memory (the scores, the lengths), so inputs written by
+ * that kernel are seen.
  */
 spattn_status spattn_select(const spattn_dims *dims, const spattn_params *params,
                             const float *scores, const int32_t *seq_lens,
