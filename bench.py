@@ -604,39 +604,51 @@ def _time_runs(run, seconds, min_runs=1, max_runs=None):
     return times
 
 
-def cpu_baseline(inp, bts, gpu_ms):
-    """The float64 oracle on this host's cores, on a bounded sample: request
-    0 (scores, selection, attention), about 10 s of runs on every core,
-    scaled to the whole step.  When one request would take more than ~10 s,
-    the sample is its KV head 0 alone (scaled by the KV heads too), and when
-    that would too (long prefill chunks), the attention of the chunk's last
-    few query tokens of KV head 0 (scaled by the tokens too).  Then a few
-    runs on one core, when they fit in ~30 s."""
+def oracle_sample(inp) -> dict:
+    """The bounded sample of a step's oracle work that both host legs time:
+    request 0 (scores, selection, attention); when one request would take
+    more than ~10 s, its KV head 0 alone; when that would too (long
+    chunks), the attention of the chunk's last few query tokens of KV head 0
+    at their own positions over the whole chunk's selection.  Returns run()
+    (-> kept block-heads of the attended heads), scale (sample -> step
+    time), kept_scale (the attended heads' kept count -> the step's), the
+    threads the sample keeps busy, and a description."""
     import oracle
 
     w = inp["workload"]
     H, Tq = w.num_kv_heads, w.q_tokens
-    cores = oracle.num_threads()
     # one query token of KV head 0: the whole unit is at most Tq times that
     t_tok = min(_time_runs(oracle_request(inp, 0, heads=[0], last_tokens=1), 0.0, min_runs=1, max_runs=1))
     t_unit = t_tok * Tq
     whole = w.hca or H == 1 or t_unit * H <= 10.0   # (the HCA branch covers every head at once)
     n_tok = Tq if t_unit <= 10.0 else max(1, min(Tq, int(10.0 / t_tok)))
-    run = oracle_request(inp, 0) if whole else oracle_request(inp, 0, heads=[0], last_tokens=n_tok)
-    scale = w.batch if whole else w.batch * H * Tq / n_tok
     what = (f"request 0 of {w.batch} (all {H} KV heads{', both branches' if w.hca else ''})" if whole
             else f"KV head 0 of request 0 (one of {w.batch * H} (request, KV head) units)" if n_tok == Tq
             else (f"the last {n_tok} of {Tq} query tokens of KV head 0 of request 0 (one of {w.batch * H} "
                   f"(request, KV head) units; selection over the whole chunk)"))
+    return {"run": oracle_request(inp, 0) if whole else oracle_request(inp, 0, heads=[0], last_tokens=n_tok),
+            "scale": w.batch if whole else w.batch * H * Tq / n_tok,
+            "kept_scale": w.batch if whole else w.batch * H,
+            # the oracle's attention runs its (request, KV head) units in parallel
+            "cores": min(oracle.num_threads(), H if whole else 1),
+            "what": what}
+
+
+def cpu_baseline(inp, bts, gpu_ms):
+    """The float64 oracle on this host's cores on the bounded sample of
+    oracle_sample(), about 10 s of runs, median scaled to the whole step;
+    then a few runs on one core, when they fit in ~30 s."""
+    import oracle
+
+    cores = oracle.num_threads()
+    smp = oracle_sample(inp)
+    run, scale, used = smp["run"], smp["scale"], smp["cores"]
     times = _time_runs(run, 10.0)
     per = statistics.median(times)
     step_s = per * scale
-    # the oracle's attention runs its (request, KV head) units in parallel:
-    # the threads the sample keeps busy
-    used = min(cores, H if whole else 1)
     line = {"value": round(bts["total"] / step_s / 1e9, 4), "unit": "GB/s", "cores": used,
             "host_threads": cores, "kind": "oracle",
-            "sample": f"{what}, {len(times)} runs, median {per:.3f} s, scaled x{scale:g} to the step",
+            "sample": f"{smp['what']}, {len(times)} runs, median {per:.3f} s, scaled x{scale:g} to the step",
             "ms_per_step": round(step_s * 1e3, 3), "gpu_speedup": round(step_s * 1e3 / gpu_ms, 1)}
     # one core: the same sample, if about 5 runs fit in ~30 s
     if per * used * 5 <= 30.0 or used == 1:
@@ -653,10 +665,10 @@ def cpu_baseline(inp, bts, gpu_ms):
 
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: rank 0 only.  One step = the oracle's
-    work for one request (all its KV heads; requests 0 and 1 in turn), on
-    every host core, scaled to the batch: the same sample as the native
-    arm's cpu_baseline.  Bounded to about 150 s of timed work."""
+    """The oracle as the reference arm: rank 0 only.  One step = one run of
+    the native arm's cpu_baseline sample (oracle_sample: request 0, or one of
+    its KV heads, or the last tokens of one, on every core), scaled to the
+    batch.  Bounded to about 150 s of timed work."""
     if rank != 0:
         return None
     import oracle
@@ -664,32 +676,33 @@ def run_reference(args, rank, world):
     w = WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(w, device=dev)
-    runs = [oracle_request(inp, b) for b in range(min(w.batch, 2))]
-    for i in range(args.warmup):
-        runs[i % len(runs)]()
+    smp = oracle_sample(inp)
+    run = smp["run"]
+    for _ in range(args.warmup):
+        run()
     times, kept = [], 0
     budget = time.perf_counter() + 150.0
-    for i in range(args.steps):
+    for _ in range(args.steps):
         t0 = time.perf_counter()
-        kept += runs[i % len(runs)]()
+        kept += run()
         times.append(time.perf_counter() - t0)
         if time.perf_counter() > budget:
             break
-    per_req = statistics.median(times)
-    step_s = per_req * w.batch
-    # bytes of a full step at the sampled requests' mean kept count
+    per = statistics.median(times)
+    step_s = per * smp["scale"]
+    # bytes of a full step at the sample's kept count
     P, D = w.block_size, w.head_dim
     elt = 1 if w.kv_fp8 else 2
-    mean_kept = kept / len(times)
+    kept_step = kept / len(times) * smp["kept_scale"]
     nbs = [(int(L) + P - 1) // P for L in inp["seq_lens"].tolist()]
     n_mid = sum(max(0, nb - w.sink_blocks - w.local_blocks) for nb in nbs)
-    total = (w.batch * mean_kept * P * D * elt * 2 + (w.batch * mean_kept * 8 if w.kv_fp8 else 0)
+    total = (kept_step * P * D * elt * 2 + (kept_step * 8 if w.kv_fp8 else 0)
              + n_mid * w.num_kv_heads * D * (2 if w.kbar_bf16 else 4) + inp["q"].numel() * 6)
     if w.hca:
         total += step_bytes(inp, torch.zeros(1))["hca"]
     value = total / step_s / 1e9
-    sample = (f"{len(times)} steps x one request of {w.batch} (all {w.num_kv_heads} KV heads: scores, selection, "
-              f"attention{', HCA branch and merge' if w.hca else ''} in float64), median scaled x{w.batch}")
+    sample = (f"{len(times)} steps x {smp['what']} (scores, selection, attention"
+              f"{', HCA branch and merge' if w.hca else ''} in float64), median scaled x{smp['scale']:g}")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
         "n_gpus": world, "steps": len(times), "warmup": args.warmup,
@@ -697,7 +710,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; power-law block importance)",
         "config": workload_config(w, world),
         "cpu_baseline": {"value": round(value, 5), "unit": "GB/s",
-                         "cores": min(oracle.num_threads(), w.num_kv_heads), "host_threads": oracle.num_threads(),
+                         "cores": smp["cores"], "host_threads": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
