@@ -1,7 +1,8 @@
-"""bench.py's algorithmic FLOP count of the sparse attention, against a
-brute-force count of (query row, visible kept token) pairs on small cases:
-decode rows (every kept token visible) and chunks (causal within the chunk,
-partly filled last block)."""
+"""bench.py's host-side accounting: the algorithmic FLOP count of the sparse
+attention against a brute-force count of (query row, visible kept token)
+pairs on small cases (decode rows see every kept token; chunk rows are
+causal within the chunk; partly filled last block), and the oracle sample
+both host legs time, with its scale to a whole step."""
 import random
 
 import torch
@@ -71,3 +72,20 @@ def test_oracle_sample_of_the_last_chunk_tokens():
     full = bench.oracle_request(inp, 0, heads=[0])()
     part = bench.oracle_request(inp, 0, heads=[0], last_tokens=3)()
     assert full == part > 0
+
+
+def test_oracle_sample_scaling(monkeypatch):
+    """The host legs' sample and its scale to the step: the whole request
+    when it is short, one KV head when the request is long, the last few
+    query tokens of one head when even that is long."""
+    from block_sparse_kv_spattn_b200.workloads import make_inputs
+    w = Workload("t", batch=3, q_tokens=8, num_q_heads=8, num_kv_heads=2, seq_len=64 * 6, structure="zipf",
+                 mode="topk", max_ratio=0.3, seed=6)
+    inp = make_inputs(w, device="cpu")
+    for t_tok, kind, scale, kept_scale in ((0.1, "request 0", 3, 3), (1.0, "KV head 0", 6, 6),
+                                           (4.0, "last 2 of 8", 24, 6)):
+        monkeypatch.setattr(bench, "_time_runs", lambda run, seconds, min_runs=1, max_runs=None, t=t_tok: [t])
+        smp = bench.oracle_sample(inp)
+        assert kind in smp["what"], smp["what"]
+        assert smp["scale"] == scale and smp["kept_scale"] == kept_scale
+        assert smp["run"]() > 0
