@@ -285,7 +285,9 @@ spattn_status launch_scores(const spattn_dims *d, const spattn_params *p, const 
     a.tt = std::max(1, std::min(d->q_tokens, 128 / d->num_kv_heads));
     const int rowsq = a.tt * d->num_kv_heads;
     const int ztiles = (d->q_tokens + a.tt - 1) / a.tt;
-    const int bpc_min = score_blocks_per_cta(rowsq);   // (a one-wave grid of more blocks per CTA measured slower)
+    // (with 8 KV heads a one-wave grid of more blocks per CTA measured slower;
+    // with one or two, faster: score_blocks_per_cta)
+    const int bpc_min = score_blocks_per_cta(rowsq);
     auto smem_of = [&](int bpc) {
         return rowsq * (kHeadDim + bpc) * (int)sizeof(float) + bpc * (int)sizeof(int);
     };
